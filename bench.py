@@ -1,0 +1,490 @@
+"""Benchmark of the normalise-then-rotate hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline workload (one step = one fused_qk_norm_rope launch over the whole
+batch): joint text/image QK RMSNorm + cat + RoPE, 512 text + 4096 image
+tokens, 24 heads, head dim 128, bf16, GPT-J pairing, fp32 [4608, 64] cos/sin
+table -- the fused op the vllm-omni page measures (256 + 4096 tokens there).
+``value`` is tokens/s over all ranks (weak scaling: every rank processes its
+own batch, no data-path collective).  Inputs rotate over several copies whose
+total exceeds twice the 126 MB L2, so every launch reads from HBM.
+
+The JSON line also carries a ``rows`` list: every other kernel of the path
+measured at its own workload (RMSNorm + residual decode and sweep points,
+interleaved mRoPE unchunked and chunked, ViT setup and apply).
+
+``--impl reference`` times the CPU oracle (single thread, the machine's host
+cores) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "fused QK-norm+RoPE tokens/s and achieved HBM GB/s (% of B200 peak) at 1 GPU"
+L2_BYTES = 126 * 2 ** 20
+WORKLOAD = "joint text/image QK RMSNorm + cat + RoPE (512 txt + 4096 img tokens, 24 heads, " \
+           "head_dim 128, bf16, GPT-J pairing, fp32 cos/sin table [4608,64])"
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return e["dram_bytes_per_launch"] if h == e["source_sha256"] else None
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        win = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples
+        mhz = [s[1] for s in win]
+        mask = 0
+        for s in win:
+            mask |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win)}
+
+
+# ------------------------------------------------------- headline (fused) --
+
+def fused_bytes(T_txt, T_img, H, D, P):
+    T = T_txt + T_img
+    qk = 2 * T * H * D * 2           # read q and k of both streams
+    out = 2 * T * H * D * 2          # write joint q and k
+    gam = 4 * D * 2
+    tab = 2 * T * P * 4              # cos and sin rows read once each
+    return qk + out + gam + tab
+
+
+class FusedSet:
+    """One full set of device inputs and outputs of the headline workload."""
+
+    def __init__(self, w, dev):
+        import mrope_qk_norm_b200 as qkr
+        self.qkr = qkr
+        self.streams = []
+        for s in w.streams:
+            self.streams.append(tuple(t.to(dev) for t in (s.q, s.k, s.gamma_q, s.gamma_k)))
+        self.cos = w.angle.cos.to(dev)
+        self.sin = w.angle.sin.to(dev)
+        T = w.n_tokens
+        self.qo = torch.empty(T, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
+        self.ko = torch.empty(T, w.Hk, w.D, dtype=torch.bfloat16, device=dev)
+        self.angle = qkr.angle_table(self.cos, self.sin)
+        self.descs = [qkr.stream_desc(*s) for s in self.streams]
+        self.w = w
+
+    def launch(self, stream=None):
+        self.qkr.fused_qk_norm_rope(self.descs, self.qo, self.ko, self.w.rot, self.w.pairing,
+                                    self.w.eps, self.angle, 0, stream)
+
+
+def time_launches(fns, steps, warmup, stream):
+    """Run fns[i % len] `steps` times; returns (total_ms, per-launch ms list)."""
+    for i in range(warmup):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        fns[i % len(fns)]()
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end), [a.elapsed_time(b) for a, b in ev]
+
+
+def n_sets_for(bytes_per_set: int) -> int:
+    return max(1, min(8, -(-2 * L2_BYTES // bytes_per_set) + 1))
+
+
+# ------------------------------------------------------------- other rows --
+
+def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20):
+    """Each remaining kernel of the path at its own workload."""
+    import mrope_qk_norm_b200 as qkr
+    rows = []
+
+    def record(name, workload, fns, nbytes, units, unit_name, extra=None):
+        total, per = time_launches(fns, steps, warmup, stream)
+        us = 1e3 * statistics.mean(per)
+        gbs = nbytes / (us * 1e-6) / 1e9
+        r = {"kernel": name, "workload": workload, "us_per_launch": round(us, 3),
+             "algorithmic_bytes": nbytes, "achieved_gbs": round(gbs, 1),
+             "frac_of_measured_hbm": round(gbs / peak_gbs, 4),
+             unit_name + "_per_s": round(units / (us * 1e-6), 1),
+             "launch": qkr.last_launch()}
+        if extra:
+            r.update(extra)
+        rows.append(r)
+
+    # config 1: single-stream, latency-bound
+    w = W.config1()
+    s = [t.to(dev) for t in (w.streams[0].q, w.streams[0].k, w.streams[0].gamma_q,
+                             w.streams[0].gamma_k)]
+    pos, inv = w.angle.positions.to(dev), w.angle.inv_freq.to(dev)
+    qo, ko = torch.empty_like(s[0]), torch.empty_like(s[1])
+    a = qkr.angle_positions(pos, inv)
+    d = [qkr.stream_desc(*s)]
+    record("fused_qk_norm_rope", "single-stream T=16 H=4 D=64 NeoX",
+           [lambda: qkr.fused_qk_norm_rope(d, qo, ko, 64, 0, 1e-6, a, 0, stream)],
+           33216, 16, "tokens")
+
+    # config 3 with NeoX pairing
+    w3n = W.config3(pairing=W.PAIRING_NEOX)
+    b3 = fused_bytes(512, 4096, 24, 128, 64)
+    sets = [FusedSet(w3n, dev) for _ in range(n_sets_for(b3))]
+    record("fused_qk_norm_rope", "joint 512+4096 tokens H=24 D=128 NeoX",
+           [lambda s=s: s.launch(stream) for s in sets], b3, 4608, "tokens")
+    del sets
+
+    # config 4: interleaved mRoPE (no norm), unchunked and chunked at 2457
+    w4 = W.config4()
+    T, Hq, Hkv, D = 8192, 16, 8, 128
+    b4 = 2 * (T * Hq * D * 2 + T * Hkv * D * 2) + 3 * T * 4 + 64 * 4
+    n4 = n_sets_for(b4)
+    s4 = []
+    for _ in range(n4):
+        q, k = w4.streams[0].q.to(dev), w4.streams[0].k.to(dev)
+        s4.append((q, k, torch.empty_like(q), torch.empty_like(k)))
+    pos4, inv4 = w4.angle.positions.to(dev), w4.angle.inv_freq.to(dev)
+
+    def mr(x, chunks):
+        q, k, qo_, ko_ = x
+        for t0, t1 in chunks:
+            qkr.mrope_apply(q[t0:t1], k[t0:t1], qo_[t0:t1], ko_[t0:t1], pos4, inv4, 128,
+                            W.SECTIONS_INTERLEAVED, (24, 20, 20), 0, token_offset=t0,
+                            stream=stream)
+    record("mrope_apply", "interleaved mRoPE T=8192 Hq=16 Hkv=8 D=128 (24,20,20)",
+           [lambda x=x: mr(x, [(0, 8192)]) for x in s4], b4, 8192, "tokens")
+    record("mrope_apply", "same, two chunked launches split at 2457 (per step)",
+           [lambda x=x: mr(x, [(0, 2457), (2457, 8192)]) for x in s4], b4, 8192, "tokens",
+           {"launches_per_step": 2})
+    del s4
+
+    # config 5: ViT setup and apply
+    w5 = W.config5()
+    g = np.asarray(w5.grids, dtype=np.int64)
+    cu = np.concatenate([[0], np.cumsum(g[:, 0] * g[:, 1] * g[:, 2])])
+    N = int(cu[-1])
+    meta = torch.from_numpy(np.concatenate([cu, g.reshape(-1)]).astype(np.int32)).to(dev)
+    G = len(w5.grids)
+    cu_d, grids_d = meta[:G + 1], meta[G + 1:].view(G, 3)
+    inv_t, inv_h, inv_w = (v.to(dev) for v in (w5.inv_t, w5.inv_h, w5.inv_w))
+    cos5 = torch.empty(3, N, 64, dtype=torch.float32, device=dev)
+    sin5 = torch.empty_like(cos5)
+    setup_bytes = 2 * N * 64 * 4 + (G + 1 + 3 * G) * 4 + 64 * 4
+    record("vit_mrope_setup", "8 grids N=%d, planes (3,N,64) fp32" % N,
+           [lambda: qkr.vit_mrope_setup(inv_t, inv_h, inv_w, cu_d, grids_d, N, 2, cos5, sin5,
+                                        stream)], setup_bytes, N, "tokens")
+    q5, k5 = w5.q.to(dev), w5.k.to(dev)
+    gq5, gk5 = w5.gamma_q.to(dev), w5.gamma_k.to(dev)
+    qo5, ko5 = torch.empty_like(q5), torch.empty_like(k5)
+    a5 = qkr.angle_table(cos5, sin5, W.SECTIONS_CONTIGUOUS, (16, 24, 24))
+    d5 = [qkr.stream_desc(q5, k5, gq5, gk5)]
+    apply_bytes = 4 * N * 16 * 80 * 2 + 2 * N * 32 * 4 + 4 * 80 * 2
+    record("fused_qk_norm_rope", "ViT apply N=%d H=16 D=80 rot=64 from the 3 planes" % N,
+           [lambda: qkr.fused_qk_norm_rope(d5, qo5, ko5, 64, 0, 1e-6, a5, 0, stream)],
+           apply_bytes, N, "tokens")
+
+    # config 2: RMSNorm + residual, decode rows and sweep points
+    for R, hidden in [(1, 5120), (32, 5120), (1024, 8192), (16384, 8192), (16384, 2048)]:
+        nb = 8 * R * hidden + 2 * hidden
+        nset = n_sets_for(nb)
+        sets = []
+        for _ in range(nset):
+            w2 = W.config2(R=R, hidden=hidden)
+            sets.append((w2.x.to(dev), w2.residual.to(dev), w2.gamma.to(dev),
+                         torch.empty(R, hidden, dtype=torch.bfloat16, device=dev)))
+        record("rms_norm_residual", "R=%d hidden=%d" % (R, hidden),
+               [lambda s=s: qkr.rms_norm_residual(s[0], s[1], s[2], s[3], 1e-6, stream)
+                for s in sets], nb, R, "rows")
+        del sets
+    torch.cuda.synchronize()
+    return rows
+
+
+# ------------------------------------------------------------- CPU oracle --
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    """The oracle as it stands, single-threaded, on a bounded token sample."""
+    import oracle
+    w = W.config3()
+    n_img = 512
+    s_txt = w.streams[0]
+    s_img = W.StreamInputs(w.streams[1].q[:n_img], w.streams[1].k[:n_img],
+                           w.streams[1].gamma_q, w.streams[1].gamma_k)
+    tokens = s_txt.q.shape[0] + n_img
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        oracle.qk_norm_rope([s_txt, s_img], 24, 24, 128, 128, w.pairing, w.eps, w.angle)
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(calls * tokens / dt, 1), "unit": "tokens/s", "cores": 1,
+            "kind": "oracle",
+            "sample": "%d calls x %d tokens (all 512 text + first %d image tokens of the "
+                      "headline workload), fp64 C oracle, one thread, %.1f s"
+                      % (calls, tokens, n_img, dt)}
+
+
+# ------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-kernel rows")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks = measured_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = cpu_baseline(budget_s=max(2.0, min(60.0, 0.25 * max(args.steps, 1))))
+        line = {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": WORKLOAD, "sample": cb["sample"]},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import mrope_qk_norm_b200 as qkr
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=dev)
+        dist = dist_mod
+    stream = torch.cuda.current_stream(dev)
+
+    w = W.config3()  # GPT-J pairing, full size
+    nbytes = fused_bytes(512, 4096, 24, 128, 64)
+    n_sets = n_sets_for(nbytes)
+    sets = [FusedSet(w, dev) for _ in range(n_sets)]
+    fns = [lambda s=s: s.launch(stream) for s in sets]
+
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else local)
+    sampler.start()
+    for i in range(args.warmup):
+        fns[i % n_sets]()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    total_ms, per = time_launches(fns, args.steps, 0, stream)
+    t_wall1 = time.perf_counter()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.stop()
+    info = qkr.last_launch()
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_max = float(t.item())
+    ms_per_step = total_max / args.steps
+    tokens = w.n_tokens
+    value = world * tokens / (ms_per_step * 1e-3)
+    kern_ms = statistics.mean(per)
+    achieved = nbytes / (kern_ms * 1e-3) / 1e9
+
+    # end to end: pinned host inputs -> device -> kernel -> pinned host outputs
+    host_in = []
+    for s in w.streams:
+        host_in += [s.q.pin_memory(), s.k.pin_memory(), s.gamma_q.pin_memory(),
+                    s.gamma_k.pin_memory()]
+    host_in += [w.angle.cos.pin_memory(), w.angle.sin.pin_memory()]
+    e2e_set = sets[0]
+    dev_in = []
+    for s in e2e_set.streams:
+        dev_in += list(s)
+    dev_in += [e2e_set.cos, e2e_set.sin]
+    host_out = [torch.empty(e2e_set.qo.shape, dtype=torch.bfloat16).pin_memory(),
+                torch.empty(e2e_set.ko.shape, dtype=torch.bfloat16).pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step():
+        for hsrc, ddst in zip(host_in, dev_in):
+            ddst.copy_(hsrc, non_blocking=True)
+        e2e_set.launch(stream)
+        host_out[0].copy_(e2e_set.qo, non_blocking=True)
+        host_out[1].copy_(e2e_set.ko, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / args.e2e_steps
+    e2e_value = world * tokens / (e2e_ms * 1e-3)
+
+    rows = []
+    if not args.no_rows:
+        del sets, fns
+        torch.cuda.empty_cache()
+        rows = measure_rows(dev, stream, peaks["hbm_gbs"])
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cb = cpu_baseline()
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    clocks = sampler.summary(t_wall0, t_wall1)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": tokens,
+                   "parallelism": "dp%d (independent batches, no collective)" % world,
+                   "l2": "%d rotating input/output sets of %.1f MB (%.0f MB > 2x126 MB L2)"
+                         % (n_sets, nbytes / 1e6, n_sets * nbytes / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": kernel_traffic("fused_qk_norm_rope_joint"),
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peaks["source"],
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "kernel_us_per_launch": round(kern_ms * 1e3, 3),
+                     "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
+                     "kernel": info.get("kernel_name")},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "path": "pinned host -> cudaMemcpyAsync -> fused_qk_norm_rope -> pinned host"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "rows": rows,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,308 @@
+/*
+ * qkr.h -- C ABI of the B200 (sm_100a) normalise-then-rotate library.
+ *
+ * Four operations, each one CUDA kernel launch on the caller's stream:
+ *
+ *   fused_qk_norm_rope  per-head RMSNorm of Q and K, optional text/image
+ *                       concatenation, RoPE (NeoX or GPT-J pairing), one launch.
+ *   mrope_apply         multi-section RoPE (contiguous or interleaved
+ *                       sections) with a token offset for chunked launches,
+ *                       optional per-head RMSNorm.
+ *   vit_mrope_setup     fp32 (3, N, P) cos/sin t/h/w planes computed from
+ *                       per-image [t, h, w] grids.
+ *   rms_norm_residual   hidden-size RMSNorm with a fused residual add; splits
+ *                       one row across a thread-block cluster when rows are few.
+ *
+ * Conventions shared by every entry point:
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Pointers marked "device" are CUDA device (or managed) memory; pointers
+ *     marked "host" are read during the call and may be freed after it returns.
+ *   - bf16 tensors are passed as void* to IEEE bfloat16 data; strides and
+ *     offsets are in elements, never bytes; all sizes are int64_t.
+ *   - The caller owns all memory.  No entry point allocates, frees or
+ *     synchronises; each enqueues its work on `stream` and returns.
+ *   - Arguments are validated on the host before anything is enqueued.  A
+ *     call that cannot be served exactly returns an error; there is no
+ *     fallback path and no silent degradation.
+ *   - A call with zero tokens (or rows) enqueues nothing and returns QKR_OK.
+ *   - Errors: QKR_ERR_INVALID_ARG (bad sizes, null pointers, inconsistent
+ *     descriptors), QKR_ERR_UNSUPPORTED (valid but outside what the kernels
+ *     serve: alignment, head_dim range, aliasing), QKR_ERR_CUDA (the launch
+ *     failed).  qkr_last_error() returns a message for the calling thread's
+ *     most recent failure.
+ *   - Results are deterministic: fixed launch shape for a given call, no
+ *     atomics, fixed reduction order.
+ */
+#ifndef QKR_H
+#define QKR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qkr_status {
+    QKR_OK = 0,
+    QKR_ERR_INVALID_ARG = 1,
+    QKR_ERR_UNSUPPORTED = 2,
+    QKR_ERR_CUDA = 3
+} qkr_status;
+
+/* Rotary pairing.  NeoX ("rotate half") pairs dim j with dim j + rot/2;
+ * GPT-J ("interleaved") pairs dim 2j with dim 2j+1 (vllm-omni #7600: the
+ * single-stream op is called with interleaved=True).  Pair j is rotated by
+ * angle theta_j: a' = a cos - b sin, b' = b cos + a sin. */
+enum { QKR_PAIRING_NEOX = 0, QKR_PAIRING_GPTJ = 1 };
+
+/* Which position row (t = 0, h = 1, w = 2, e = 3) each rotated pair j < P
+ * reads.  sections[] = {s_t, s_h, s_w, s_e}.
+ *   NONE                every pair reads row 0 (plain 1-D RoPE).
+ *   CONTIGUOUS          pairs [0,s_t) -> t, [s_t, s_t+s_h) -> h, rest -> w
+ *                       (vLLM mrope_vit_setup: section columns of the planes).
+ *   INTERLEAVED         pair j -> j mod 3 while j < 3*min(s_t,s_h,s_w),
+ *                       else the axis of its contiguous section.
+ *   INTERLEAVED_QUOTA   same head; each later pair goes to the first axis
+ *                       (t, h, w order) whose section count is not used up.
+ *   IMROPE              llama.cpp fork #286 sector rule: sector = j mod
+ *                       (s_t+s_h+s_w+s_e); sector mod 3 == 1 -> h while
+ *                       sector < 3*s_h, == 2 -> w while < 3*s_w, == 0 -> t
+ *                       while < 3*s_t, otherwise e.  Needs four rows.
+ * Admission (llama.cpp fork #286, review of the claim predicate): for every
+ * mode but NONE, each section >= 0 and P <= sum(sections) <= 2P; s_e must be
+ * 0 unless the mode is IMROPE. */
+enum {
+    QKR_SECTIONS_NONE = 0,
+    QKR_SECTIONS_CONTIGUOUS = 1,
+    QKR_SECTIONS_INTERLEAVED = 2,
+    QKR_SECTIONS_INTERLEAVED_QUOTA = 3,
+    QKR_SECTIONS_IMROPE = 4
+};
+
+/* Where the cos/sin of pair j for a token come from. */
+enum {
+    /* theta = fp32(pos) * inv_freq[j] (one fp32 multiply), cos/sin by the
+     * accurate single-precision sincos; pos = positions[row(j) *
+     * pos_row_stride + token_offset + t] (vLLM mrope_vit_setup kernel: fp32
+     * position times fp32 inverse frequency). */
+    QKR_ANGLE_POSITIONS = 0,
+    /* cos/sin read from fp32 tables: element [plane(j)][token_offset + t][j]
+     * at plane(j) * plane_stride + (token_offset + t) * ld + j.  With
+     * QKR_SECTIONS_NONE this is the single packed table of vllm-omni #7600
+     * (one [cos | sin] table per forward); with CONTIGUOUS it reads the
+     * (3, N, P) planes written by vit_mrope_setup. */
+    QKR_ANGLE_TABLE = 1
+};
+
+/* Flags for fused_qk_norm_rope / mrope_apply. */
+enum {
+    /* Round the normalised value to bf16 before rotating (the rounding
+     * contract of the vllm-omni #7600 Triton tile: bf16-rounded normalised
+     * value, fp32 rotation, one final rounding).  Without the flag every
+     * intermediate stays in fp32 and only the output is rounded. */
+    QKR_FLAG_ROUND_NORMALIZED_BF16 = 1u
+};
+
+/* One input stream of fused_qk_norm_rope.  q and k are bf16 device pointers;
+ * element (t, h, d) of Q is at q + q_offset + t*q_tok_stride +
+ * h*q_head_stride + d (d contiguous), likewise K.  Offsets may exceed 2^31
+ * elements: all address arithmetic is 64-bit (vllm-omni #7600, 64-bit row
+ * addressing for large storage offsets).  gamma_q / gamma_k: bf16 [D] device. */
+typedef struct qkr_stream_desc {
+    const void *q;
+    const void *k;
+    int64_t q_offset;
+    int64_t k_offset;
+    int64_t q_tok_stride;
+    int64_t q_head_stride;
+    int64_t k_tok_stride;
+    int64_t k_head_stride;
+    int64_t n_tokens;
+    const void *gamma_q;
+    const void *gamma_k;
+} qkr_stream_desc;
+
+/* Angle source (see QKR_ANGLE_*).  Unused fields are ignored.
+ *   positions      device int32 [rows, pos_row_stride]; rows = 1 (NONE),
+ *                  3 (CONTIGUOUS / INTERLEAVED*), 4 (IMROPE).
+ *   pos_row_stride elements between rows = tokens the buffer covers
+ *                  (llama.cpp fork #286: a chunk keeps the whole positions
+ *                  buffer and is told where its tokens start).
+ *   inv_freq       device fp32 [P], P = rot_dim / 2.
+ *   cos, sin       device fp32 tables; table_rows tokens per plane, ld >= P
+ *                  elements between token rows, plane_stride elements
+ *                  between planes (planes: 1 for NONE, 3 for CONTIGUOUS and
+ *                  INTERLEAVED*, 4 for IMROPE).
+ *   token_offset   added to the launch-local token index before the
+ *                  positions / tables are indexed; token_offset + tokens
+ *                  of the launch must not exceed pos_row_stride (table_rows).
+ */
+typedef struct qkr_angle_desc {
+    int32_t kind;
+    int32_t section_mode;
+    int32_t sections[4];
+    const int32_t *positions;
+    int64_t pos_row_stride;
+    const float *inv_freq;
+    const float *cos;
+    const float *sin;
+    int64_t table_rows;
+    int64_t ld;
+    int64_t plane_stride;
+    int64_t token_offset;
+} qkr_angle_desc;
+
+/*
+ * fused_qk_norm_rope -- vllm-omni #7600 ("Fuse text/image QK RMSNorm + cat +
+ * RoPE into one Triton launch", Purpose and the kernel review): for every
+ * token and head, y = x / sqrt(mean(x^2) + eps) * gamma over the head dim
+ * (fp32 sum of squares), then RoPE on the first rot_dim dims; dims
+ * [rot_dim, D) are normalised only.  With n_streams == 2 the streams are
+ * concatenated text first: stream 0's tokens occupy joint rows
+ * [0, T0), stream 1's [T0, T0+T1), and the angle of joint row n is that of
+ * token token_offset + n.
+ *
+ *   streams          host array of n_streams (1 or 2) descriptors.
+ *   q_out, k_out     bf16 device [T0+T1, Hq, D] and [T0+T1, Hk, D]; row n
+ *                    of Q starts at q_out + n*q_out_tok_stride (heads dense).
+ *                    Fresh outputs: they must not overlap any input.
+ *   D                head dim, a multiple of 8, 8 <= D <= 256.
+ *   rot_dim          even, 0 <= rot_dim <= D.
+ *   flags            0 or QKR_FLAG_ROUND_NORMALIZED_BF16.
+ * Alignment: q/k (after offsets), gammas and outputs 16-byte aligned; all
+ * token and head strides multiples of 8 elements (else QKR_ERR_UNSUPPORTED).
+ */
+qkr_status fused_qk_norm_rope(void *stream, const qkr_stream_desc *streams, int32_t n_streams,
+                              void *q_out, void *k_out, int64_t q_out_tok_stride,
+                              int64_t k_out_tok_stride, int64_t Hq, int64_t Hk, int64_t D,
+                              int64_t rot_dim, int32_t pairing, float eps,
+                              const qkr_angle_desc *angle, uint32_t flags);
+
+/*
+ * mrope_apply -- multi-section RoPE (llama.cpp fork #286, "The change":
+ * each rotated pair reads the position section its index selects; a launch
+ * over a token chunk keeps the whole positions buffer and is told where its
+ * tokens start).  Rotates Q [T, Hq, D] and K [T, Hkv, D] (heads dense, token
+ * strides given) with angles from positions + inv_freq, pair j reading row
+ * section(j) at column token_offset + t.  If gamma_q and gamma_k are both
+ * non-NULL each head is RMS-normalised first (as fused_qk_norm_rope); both
+ * NULL means no normalisation; one NULL is an error.
+ *
+ *   q, k             bf16 device inputs; q_out, k_out bf16 device outputs.
+ *                    In-place is allowed: q_out == q with the same token
+ *                    stride (likewise k); any other overlap is refused.
+ *   positions        device int32 [n_rows, T_total]; n_rows must match the
+ *                    section mode (1 NONE, 3 sectioned, 4 IMROPE).
+ *   token_offset     first token of this launch within positions;
+ *                    token_offset + T <= T_total.
+ *   inv_freq         device fp32 [rot_dim / 2].
+ *   sections         host int32[4] {s_t, s_h, s_w, s_e} (may be NULL for
+ *                    QKR_SECTIONS_NONE; NULL with any other mode is an error).
+ * Same D / rot_dim / alignment rules as fused_qk_norm_rope.
+ */
+qkr_status mrope_apply(void *stream, const void *q, const void *k, void *q_out, void *k_out,
+                       int64_t T, int64_t Hq, int64_t Hkv, int64_t D, int64_t rot_dim,
+                       int64_t q_tok_stride, int64_t k_tok_stride, int64_t q_out_tok_stride,
+                       int64_t k_out_tok_stride, const int32_t *positions, int64_t n_rows,
+                       int64_t T_total, int64_t token_offset, const float *inv_freq,
+                       const int32_t *sections, int32_t section_mode, int32_t pairing,
+                       const void *gamma_q, const void *gamma_k, float eps, uint32_t flags);
+
+/*
+ * vit_mrope_setup -- vLLM mrope_vit_setup (VitMropeSetup.forward and
+ * _vit_mrope_setup_kernel): the (3, N, P) fp32 cos/sin t/h/w planes,
+ * P = half_t + half_h + half_w.  Token n of grid g (cu_seqlens[g] <= n <
+ * cu_seqlens[g+1], grid [t, h, w]) has local index l = n - cu_seqlens[g];
+ * frames hold h*w tokens ordered by spatial-merge block: merge-block row,
+ * merge-block column, then the m x m patch in row-major order, so
+ * t_pos = l / (h*w), h_pos = block_row*m + patch_row, w_pos = block_col*m +
+ * patch_col.  Plane a holds, in its own section columns only ([0, half_t)
+ * for t, [half_t, half_t+half_h) for h, the rest for w),
+ * cos/sin(fp32(pos_a) * inv_a[col - offset_a]); other columns are not
+ * written.
+ *
+ *   inv_t/h/w        device fp32 [half_t], [half_h], [half_w].
+ *   cu_seqlens       device int32 [G+1], nondecreasing, cu[0] = 0,
+ *                    cu[G] = N (the caller uploads it with grids in one copy).
+ *   grids            device int32 [G, 3] (t, h, w); h and w multiples of
+ *                    spatial_merge (not checked on the device; a violating
+ *                    grid yields positions but never an out-of-bounds access).
+ *   cos_out, sin_out device fp32 [3, N, P], 4-byte aligned.
+ */
+qkr_status vit_mrope_setup(void *stream, const float *inv_t, const float *inv_h,
+                           const float *inv_w, int64_t half_t, int64_t half_h, int64_t half_w,
+                           const int32_t *cu_seqlens, const int32_t *grids, int64_t G, int64_t N,
+                           int64_t spatial_merge, float *cos_out, float *sin_out);
+
+/*
+ * rms_norm_residual -- hidden-size RMSNorm with fused residual add
+ * (vllm.cpp #185, "decode RmsNorm ran on ONE workgroup"; vLLM #26234
+ * rms_norm_kernel): per row, s = bf16(x + residual) is written back to
+ * residual, then out = s / sqrt(mean(s^2) + eps) * gamma (fp32 sum of
+ * squares, one final bf16 rounding).  When rows are too few to fill the GPU
+ * (a single decode row) each row is split across a thread-block cluster of
+ * up to 16 CTAs whose partial sums meet in distributed shared memory.
+ *
+ *   x                bf16 device [R, hidden], row stride x_stride.
+ *   residual         bf16 device [R, hidden], in/out, row stride res_stride.
+ *   gamma            bf16 device [hidden].
+ *   out              bf16 device [R, hidden], row stride out_stride; may be
+ *                    x itself (same stride); must not overlap residual.
+ *   hidden           multiple of 8, 8 <= hidden <= 65536.
+ * Alignment: pointers 16-byte aligned, strides multiples of 8 elements.
+ */
+qkr_status rms_norm_residual(void *stream, const void *x, void *residual, const void *gamma,
+                             void *out, int64_t R, int64_t hidden, int64_t x_stride,
+                             int64_t res_stride, int64_t out_stride, float eps);
+
+/* ------------------------------------------------------------------------
+ * Introspection and debug entry points (used by the tests).
+ * ------------------------------------------------------------------------ */
+
+/* Message for the calling thread's most recent failed call ("" if none). */
+const char *qkr_last_error(void);
+
+/* Library version string. */
+const char *qkr_version(void);
+
+/* What the calling thread's most recent successful call enqueued, in the
+ * spirit of vllm.cpp #185's dispatch histogram (which kernel, what shape). */
+enum {
+    QKR_KERNEL_NONE = 0,
+    QKR_KERNEL_ROPE_PAIRED = 1,    /* NeoX, rot_dim % 16 == 0: lane holds both halves */
+    QKR_KERNEL_ROPE_VECTOR = 2,    /* GPT-J: pairs inside a lane's vector */
+    QKR_KERNEL_ROPE_EXCHANGE = 3,  /* NeoX with rot_dim % 16 != 0: shared-memory partner */
+    QKR_KERNEL_VIT_SETUP = 4,
+    QKR_KERNEL_RMS_ROWS = 5,       /* one CTA per row */
+    QKR_KERNEL_RMS_CLUSTER = 6,    /* one cluster per row */
+    QKR_KERNEL_SECTION_MAP = 7,
+    QKR_KERNEL_VIT_POSITIONS = 8
+};
+typedef struct qkr_launch_info {
+    int32_t kernel;          /* QKR_KERNEL_* */
+    int32_t lanes_per_row;   /* rope kernels: lanes that share one head row */
+    int32_t slots;           /* rope: 16-byte vectors per lane per row; rms: per thread */
+    int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
+    int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
+    int32_t block;           /* threads per CTA */
+    int64_t grid;            /* CTAs launched */
+    int64_t launches;        /* kernel launches enqueued (0 for an empty call) */
+} qkr_launch_info;
+qkr_status qkr_last_launch(qkr_launch_info *info);
+
+/* Writes the axis (0 t, 1 h, 2 w, 3 e) of pairs 0..P-1 under a section mode
+ * to axis_out (device int8 [P]) with the kernels' own section rule.
+ * sections: host int32[4].  Same admission rules as mrope_apply. */
+qkr_status qkr_section_map(void *stream, int32_t section_mode, const int32_t *sections,
+                           int64_t P, int8_t *axis_out);
+
+/* Writes the (t, h, w) position of every token to pos_out (device int32
+ * [3, N]) with vit_mrope_setup's own grid-to-position mapping. */
+qkr_status qkr_vit_positions(void *stream, const int32_t *cu_seqlens, const int32_t *grids,
+                             int64_t G, int64_t N, int64_t spatial_merge, int32_t *pos_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKR_H */

@@ -1,0 +1,563 @@
+// qkr_api.cu -- the C ABI of include/qkr.h: host-side validation and launch.
+//
+// Every entry point validates all arguments before enqueuing anything and
+// refuses (never degrades) when it cannot serve a call exactly; it never
+// allocates, frees or synchronises.
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "qkr_internal.cuh"
+
+namespace {
+
+thread_local std::string g_error;
+thread_local qkr::LaunchRecord g_last;
+
+qkr_status fail(qkr_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_error = buf;
+    return st;
+}
+
+qkr_status cuda_result(cudaError_t e, const char *what)
+{
+    if (e != cudaSuccess)
+        return fail(QKR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    g_error.clear();
+    return QKR_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Byte span [lo, hi) touched by a [T, H, D] bf16 view with positive strides.
+struct Span {
+    uintptr_t lo = 0, hi = 0;
+};
+Span view_span(const void *base, int64_t T, int64_t ts, int64_t H, int64_t hs, int64_t D)
+{
+    Span s;
+    if (T <= 0 || H <= 0)
+        return s;
+    s.lo = reinterpret_cast<uintptr_t>(base);
+    const int64_t last = (T - 1) * ts + (H - 1) * hs + D;  // elements
+    s.hi = s.lo + (uintptr_t)last * 2u;
+    return s;
+}
+bool overlap(const Span &a, const Span &b)
+{
+    return a.lo < a.hi && b.lo < b.hi && a.lo < b.hi && b.lo < a.hi;
+}
+
+// Largest element offset a view reaches must stay far from int64 overflow.
+bool view_fits(int64_t T, int64_t ts, int64_t H, int64_t hs, int64_t D)
+{
+    const __int128 last = (__int128)(T > 0 ? T - 1 : 0) * ts + (__int128)(H > 0 ? H - 1 : 0) * hs + D;
+    return last < ((__int128)1 << 60);
+}
+
+int rows_for_mode(int mode)
+{
+    return mode == QKR_SECTIONS_NONE ? 1 : (mode == QKR_SECTIONS_IMROPE ? 4 : 3);
+}
+
+qkr_status check_sections(int mode, const int32_t *sec, int64_t P, int (&out)[4])
+{
+    for (int i = 0; i < 4; ++i)
+        out[i] = 0;
+    if (mode < QKR_SECTIONS_NONE || mode > QKR_SECTIONS_IMROPE)
+        return fail(QKR_ERR_INVALID_ARG, "unknown section mode %d", mode);
+    if (mode == QKR_SECTIONS_NONE)
+        return QKR_OK;
+    if (!sec)
+        return fail(QKR_ERR_INVALID_ARG,
+                    "section mode %d needs its sections: refusing rather than rotating every "
+                    "pair by one row", mode);
+    int64_t sum = 0;
+    for (int i = 0; i < 4; ++i) {
+        if (sec[i] < 0 || sec[i] > (1 << 20))
+            return fail(QKR_ERR_INVALID_ARG, "section %d = %d out of range", i, sec[i]);
+        sum += sec[i];
+        out[i] = sec[i];
+    }
+    if (mode != QKR_SECTIONS_IMROPE && sec[3] != 0)
+        return fail(QKR_ERR_INVALID_ARG, "a fourth section is only read by the IMROPE mode");
+    if (P > 0 && (sum < P || sum > 2 * P))
+        return fail(QKR_ERR_INVALID_ARG,
+                    "sections sum to %lld; %lld rotated pairs need P <= sum <= 2P",
+                    (long long)sum, (long long)P);
+    if (P == 0 && sum == 0 && mode == QKR_SECTIONS_IMROPE)
+        return fail(QKR_ERR_INVALID_ARG, "IMROPE sections must not all be zero");
+    return QKR_OK;
+}
+
+// Angle descriptor checks; fills the device-side fields of RopeParams.
+qkr_status check_angle(const qkr_angle_desc *a, int64_t P, int64_t T, qkr::RopeParams &p)
+{
+    if (!a)
+        return fail(QKR_ERR_INVALID_ARG, "angle descriptor is NULL");
+    int sec[4];
+    qkr_status st = check_sections(a->section_mode, a->sections, P, sec);
+    if (st != QKR_OK)
+        return st;
+    p.section_mode = a->section_mode;
+    for (int i = 0; i < 4; ++i)
+        p.sec[i] = sec[i];
+    p.angle_kind = a->kind;
+    p.token_offset = a->token_offset;
+    if (a->token_offset < 0)
+        return fail(QKR_ERR_INVALID_ARG, "token_offset must be >= 0");
+    if (P == 0)
+        return QKR_OK;  // nothing is rotated: the angle source is never read
+    if (a->kind == QKR_ANGLE_POSITIONS) {
+        if (!a->positions || !a->inv_freq)
+            return fail(QKR_ERR_INVALID_ARG, "positions and inv_freq must be non-NULL");
+        if (!aligned4(a->positions) || !aligned4(a->inv_freq))
+            return fail(QKR_ERR_UNSUPPORTED, "positions / inv_freq must be 4-byte aligned");
+        if (a->pos_row_stride < 0 || a->token_offset + T > a->pos_row_stride)
+            return fail(QKR_ERR_INVALID_ARG,
+                        "token_offset (%lld) + tokens (%lld) exceeds the positions row length "
+                        "(%lld)", (long long)a->token_offset, (long long)T,
+                        (long long)a->pos_row_stride);
+        p.pos = a->positions;
+        p.pos_rs = a->pos_row_stride;
+        p.inv_freq = a->inv_freq;
+    } else if (a->kind == QKR_ANGLE_TABLE) {
+        if (!a->cos || !a->sin)
+            return fail(QKR_ERR_INVALID_ARG, "cos and sin tables must be non-NULL");
+        if (!aligned4(a->cos) || !aligned4(a->sin))
+            return fail(QKR_ERR_UNSUPPORTED, "cos / sin tables must be 4-byte aligned");
+        if (a->ld < P)
+            return fail(QKR_ERR_INVALID_ARG, "table ld (%lld) < rotated pairs (%lld)",
+                        (long long)a->ld, (long long)P);
+        if (a->table_rows < 0 || a->token_offset + T > a->table_rows)
+            return fail(QKR_ERR_INVALID_ARG,
+                        "token_offset (%lld) + tokens (%lld) exceeds the table rows (%lld)",
+                        (long long)a->token_offset, (long long)T, (long long)a->table_rows);
+        const int planes = rows_for_mode(a->section_mode);
+        if (planes > 1 && a->plane_stride < a->table_rows * a->ld)
+            return fail(QKR_ERR_INVALID_ARG, "plane_stride (%lld) smaller than one plane",
+                        (long long)a->plane_stride);
+        p.cos = a->cos;
+        p.sin = a->sin;
+        p.ld = a->ld;
+        p.plane_stride = a->plane_stride;
+    } else {
+        return fail(QKR_ERR_INVALID_ARG, "unknown angle kind %d", a->kind);
+    }
+    return QKR_OK;
+}
+
+qkr_status check_geometry(int64_t Hq, int64_t Hk, int64_t D, int64_t rot, int32_t pairing,
+                          float eps)
+{
+    if (Hq < 1 || Hk < 1 || Hq + Hk > 65536)
+        return fail(QKR_ERR_INVALID_ARG, "head counts must be >= 1 and Hq + Hk <= 65536");
+    if (D < 8 || D > 256 || D % 8)
+        return fail(QKR_ERR_UNSUPPORTED, "head_dim %lld: need a multiple of 8 in [8, 256]",
+                    (long long)D);
+    if (rot < 0 || rot > D || rot % 2)
+        return fail(QKR_ERR_INVALID_ARG, "rot_dim %lld: need an even value in [0, head_dim]",
+                    (long long)rot);
+    if (pairing != QKR_PAIRING_NEOX && pairing != QKR_PAIRING_GPTJ)
+        return fail(QKR_ERR_INVALID_ARG, "unknown pairing %d", pairing);
+    if (!(eps >= 0.f) || eps > 1.f)
+        return fail(QKR_ERR_INVALID_ARG, "eps must be finite and in [0, 1]");
+    return QKR_OK;
+}
+
+// Shared body of fused_qk_norm_rope and mrope_apply.  `inplace_ok` admits
+// outputs equal to the inputs with identical strides (mrope_apply).
+qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_streams,
+                     void *q_out, void *k_out, int64_t qo_ts, int64_t ko_ts, int64_t Hq,
+                     int64_t Hk, int64_t D, int64_t rot, int32_t pairing, float eps,
+                     const qkr_angle_desc *angle, uint32_t flags, bool norm, bool inplace_ok)
+{
+    qkr_status st = check_geometry(Hq, Hk, D, rot, pairing, eps);
+    if (st != QKR_OK)
+        return st;
+    if (!streams || n_streams < 1 || n_streams > 2)
+        return fail(QKR_ERR_INVALID_ARG, "need 1 or 2 stream descriptors");
+    if (flags & ~(uint32_t)QKR_FLAG_ROUND_NORMALIZED_BF16)
+        return fail(QKR_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    int64_t T_all = 0;
+    for (int s = 0; s < n_streams; ++s) {
+        if (streams[s].n_tokens < 0 || streams[s].n_tokens > ((int64_t)1 << 40))
+            return fail(QKR_ERR_INVALID_ARG, "stream %d: token count out of range", s);
+        T_all += streams[s].n_tokens;
+    }
+    if (T_all == 0) {  // nothing to do: enqueue nothing
+        g_last = qkr::LaunchRecord();
+        g_error.clear();
+        return QKR_OK;
+    }
+    if (!q_out || !k_out)
+        return fail(QKR_ERR_INVALID_ARG, "q_out and k_out must be non-NULL");
+    if (!aligned16(q_out) || !aligned16(k_out))
+        return fail(QKR_ERR_UNSUPPORTED, "outputs must be 16-byte aligned");
+    if (qo_ts < Hq * D || ko_ts < Hk * D || qo_ts % 8 || ko_ts % 8)
+        return fail(QKR_ERR_UNSUPPORTED,
+                    "output token strides must be multiples of 8 and hold a token's heads");
+
+    qkr::RopeParams p = {};
+    int64_t T = 0;
+    const __nv_bfloat16 *qb[2] = {nullptr, nullptr}, *kb[2] = {nullptr, nullptr};
+    for (int s = 0; s < n_streams; ++s) {
+        const qkr_stream_desc &d = streams[s];
+        if (d.n_tokens < 0)
+            return fail(QKR_ERR_INVALID_ARG, "stream %d: negative token count", s);
+        if (d.n_tokens == 0) {
+            qb[s] = kb[s] = nullptr;
+            p.st[s] = qkr::RopeStreamDev{};
+            continue;
+        }
+        if (!d.q || !d.k)
+            return fail(QKR_ERR_INVALID_ARG, "stream %d: q and k must be non-NULL", s);
+        if (d.q_offset < 0 || d.k_offset < 0)
+            return fail(QKR_ERR_INVALID_ARG, "stream %d: storage offsets must be >= 0", s);
+        if (d.q_tok_stride <= 0 || d.k_tok_stride <= 0 || d.q_head_stride < D ||
+            d.k_head_stride < D)
+            return fail(QKR_ERR_UNSUPPORTED,
+                        "stream %d: strides must be positive and heads must not overlap", s);
+        if (d.q_tok_stride % 8 || d.k_tok_stride % 8 || d.q_head_stride % 8 ||
+            d.k_head_stride % 8 || d.q_offset % 8 || d.k_offset % 8)
+            return fail(QKR_ERR_UNSUPPORTED,
+                        "stream %d: offsets and strides must be multiples of 8 elements "
+                        "(16-byte vectors)", s);
+        if (!view_fits(d.n_tokens, d.q_tok_stride, Hq, d.q_head_stride, D) ||
+            !view_fits(d.n_tokens, d.k_tok_stride, Hk, d.k_head_stride, D) ||
+            d.q_offset > ((int64_t)1 << 60) || d.k_offset > ((int64_t)1 << 60))
+            return fail(QKR_ERR_INVALID_ARG, "stream %d: view exceeds the address range", s);
+        qb[s] = static_cast<const __nv_bfloat16 *>(d.q) + d.q_offset;
+        kb[s] = static_cast<const __nv_bfloat16 *>(d.k) + d.k_offset;
+        if (!aligned16(qb[s]) || !aligned16(kb[s]))
+            return fail(QKR_ERR_UNSUPPORTED, "stream %d: q/k must be 16-byte aligned", s);
+        if (norm) {
+            if (!d.gamma_q || !d.gamma_k)
+                return fail(QKR_ERR_INVALID_ARG, "stream %d: gamma_q and gamma_k are required",
+                            s);
+            if (!aligned16(d.gamma_q) || !aligned16(d.gamma_k))
+                return fail(QKR_ERR_UNSUPPORTED, "stream %d: gammas must be 16-byte aligned", s);
+        }
+        p.st[s].q = qb[s];
+        p.st[s].k = kb[s];
+        p.st[s].q_ts = d.q_tok_stride;
+        p.st[s].q_hs = d.q_head_stride;
+        p.st[s].k_ts = d.k_tok_stride;
+        p.st[s].k_hs = d.k_head_stride;
+        p.st[s].gq = static_cast<const __nv_bfloat16 *>(d.gamma_q);
+        p.st[s].gk = static_cast<const __nv_bfloat16 *>(d.gamma_k);
+        T += d.n_tokens;
+    }
+    if (T > ((int64_t)1 << 40))
+        return fail(QKR_ERR_INVALID_ARG, "token count too large");
+    if (!view_fits(T, qo_ts, 1, 0, Hq * D) || !view_fits(T, ko_ts, 1, 0, Hk * D))
+        return fail(QKR_ERR_INVALID_ARG, "output view exceeds the address range");
+
+    // Aliasing: outputs may equal inputs only where allowed, never overlap otherwise.
+    const Span so_q = view_span(q_out, T, qo_ts, Hq, D, D);
+    const Span so_k = view_span(k_out, T, ko_ts, Hk, D, D);
+    if (overlap(so_q, so_k))
+        return fail(QKR_ERR_UNSUPPORTED, "q_out and k_out overlap");
+    for (int s = 0; s < n_streams; ++s) {
+        const qkr_stream_desc &d = streams[s];
+        if (d.n_tokens == 0)
+            continue;
+        const Span si_q = view_span(qb[s], d.n_tokens, d.q_tok_stride, Hq, d.q_head_stride, D);
+        const Span si_k = view_span(kb[s], d.n_tokens, d.k_tok_stride, Hk, d.k_head_stride, D);
+        const bool q_same = inplace_ok && n_streams == 1 && qb[s] == q_out &&
+                            d.q_tok_stride == qo_ts && d.q_head_stride == D;
+        const bool k_same = inplace_ok && n_streams == 1 && kb[s] == k_out &&
+                            d.k_tok_stride == ko_ts && d.k_head_stride == D;
+        if ((overlap(so_q, si_q) && !q_same) || overlap(so_q, si_k) ||
+            (overlap(so_k, si_k) && !k_same) || overlap(so_k, si_q))
+            return fail(QKR_ERR_UNSUPPORTED,
+                        inplace_ok ? "outputs overlap inputs (only exact in-place is allowed)"
+                                   : "outputs must not overlap the inputs (fresh outputs)");
+    }
+
+    const int64_t P = rot / 2;
+    st = check_angle(angle, P, T, p);
+    if (st != QKR_OK)
+        return st;
+
+    p.split = n_streams == 2 ? streams[0].n_tokens : INT64_MAX;
+    if (n_streams == 2 && streams[0].n_tokens == 0)
+        p.split = 0;
+    p.q_out = static_cast<__nv_bfloat16 *>(q_out);
+    p.k_out = static_cast<__nv_bfloat16 *>(k_out);
+    p.qo_ts = qo_ts;
+    p.ko_ts = ko_ts;
+    p.T = T;
+    p.Hq = (int)Hq;
+    p.Hk = (int)Hk;
+    p.D = (int)D;
+    p.rot = (int)rot;
+    p.P = (int)P;
+    p.rows_per_token = (int)(Hq + Hk);
+    p.eps = eps;
+    p.inv_D = 1.0f / (float)D;
+    p.norm = norm ? 1 : 0;
+    p.round_norm = (flags & QKR_FLAG_ROUND_NORMALIZED_BF16) ? 1 : 0;
+
+    qkr::LaunchRecord rec;
+    cudaError_t e = qkr::launch_rope_rows(p, pairing, static_cast<cudaStream_t>(stream), &rec);
+    qkr_status r = cuda_result(e, "rope kernel launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *qkr_last_error(void) { return g_error.c_str(); }
+
+const char *qkr_version(void) { return "qkr 0.1.0 (sm_100a)"; }
+
+qkr_status qkr_last_launch(qkr_launch_info *info)
+{
+    if (!info)
+        return fail(QKR_ERR_INVALID_ARG, "info is NULL");
+    info->kernel = g_last.kernel;
+    info->lanes_per_row = g_last.lanes_per_row;
+    info->slots = g_last.slots;
+    info->tokens_per_cta = g_last.tokens_per_cta;
+    info->cluster = g_last.cluster;
+    info->block = g_last.block;
+    info->grid = g_last.grid;
+    info->launches = g_last.launches;
+    return QKR_OK;
+}
+
+qkr_status fused_qk_norm_rope(void *stream, const qkr_stream_desc *streams, int32_t n_streams,
+                              void *q_out, void *k_out, int64_t q_out_tok_stride,
+                              int64_t k_out_tok_stride, int64_t Hq, int64_t Hk, int64_t D,
+                              int64_t rot_dim, int32_t pairing, float eps,
+                              const qkr_angle_desc *angle, uint32_t flags)
+{
+    return rope_call(stream, streams, n_streams, q_out, k_out, q_out_tok_stride,
+                     k_out_tok_stride, Hq, Hk, D, rot_dim, pairing, eps, angle, flags,
+                     /*norm=*/true, /*inplace_ok=*/false);
+}
+
+qkr_status mrope_apply(void *stream, const void *q, const void *k, void *q_out, void *k_out,
+                       int64_t T, int64_t Hq, int64_t Hkv, int64_t D, int64_t rot_dim,
+                       int64_t q_tok_stride, int64_t k_tok_stride, int64_t q_out_tok_stride,
+                       int64_t k_out_tok_stride, const int32_t *positions, int64_t n_rows,
+                       int64_t T_total, int64_t token_offset, const float *inv_freq,
+                       const int32_t *sections, int32_t section_mode, int32_t pairing,
+                       const void *gamma_q, const void *gamma_k, float eps, uint32_t flags)
+{
+    if ((gamma_q == nullptr) != (gamma_k == nullptr))
+        return fail(QKR_ERR_INVALID_ARG, "gamma_q and gamma_k must be both set or both NULL");
+    const bool norm = gamma_q != nullptr;
+    if (!norm && (flags & QKR_FLAG_ROUND_NORMALIZED_BF16))
+        return fail(QKR_ERR_INVALID_ARG, "ROUND_NORMALIZED_BF16 needs normalisation (gammas)");
+    if (section_mode < QKR_SECTIONS_NONE || section_mode > QKR_SECTIONS_IMROPE)
+        return fail(QKR_ERR_INVALID_ARG, "unknown section mode %d", section_mode);
+    if (rot_dim > 0 && n_rows != rows_for_mode(section_mode))
+        return fail(QKR_ERR_INVALID_ARG, "section mode %d reads %d position rows, got %lld",
+                    section_mode, rows_for_mode(section_mode), (long long)n_rows);
+    qkr_stream_desc d = {};
+    d.q = q;
+    d.k = k;
+    d.q_tok_stride = q_tok_stride;
+    d.q_head_stride = D;
+    d.k_tok_stride = k_tok_stride;
+    d.k_head_stride = D;
+    d.n_tokens = T;
+    d.gamma_q = gamma_q;
+    d.gamma_k = gamma_k;
+    qkr_angle_desc a = {};
+    a.kind = QKR_ANGLE_POSITIONS;
+    a.section_mode = section_mode;
+    if (sections)
+        for (int i = 0; i < 4; ++i)
+            a.sections[i] = sections[i];
+    a.positions = positions;
+    a.pos_row_stride = T_total;
+    a.inv_freq = inv_freq;
+    a.token_offset = token_offset;
+    if (section_mode != QKR_SECTIONS_NONE && !sections)
+        return fail(QKR_ERR_INVALID_ARG,
+                    "section mode %d needs its sections: refusing rather than rotating every "
+                    "pair by one row", section_mode);
+    return rope_call(stream, &d, 1, q_out, k_out, q_out_tok_stride, k_out_tok_stride, Hq, Hkv,
+                     D, rot_dim, pairing, eps, &a, flags, norm, /*inplace_ok=*/true);
+}
+
+static qkr_status vit_common(const int32_t *cu, const int32_t *grids, int64_t G, int64_t N,
+                             int64_t m, qkr::VitParams &p)
+{
+    if (G < 0 || N < 0)
+        return fail(QKR_ERR_INVALID_ARG, "G and N must be >= 0");
+    if (G > (1 << 24) || N > ((int64_t)1 << 40))
+        return fail(QKR_ERR_INVALID_ARG, "G or N too large");
+    if (G == 0 && N != 0)
+        return fail(QKR_ERR_INVALID_ARG, "N = %lld tokens with no grids", (long long)N);
+    if (m < 1 || m > 64)
+        return fail(QKR_ERR_INVALID_ARG, "spatial_merge must be in [1, 64]");
+    if (N > 0 && (!cu || !grids))
+        return fail(QKR_ERR_INVALID_ARG, "cu_seqlens and grids must be non-NULL");
+    if (N > 0 && (!aligned4(cu) || !aligned4(grids)))
+        return fail(QKR_ERR_UNSUPPORTED, "cu_seqlens / grids must be 4-byte aligned");
+    p.cu = cu;
+    p.grids = grids;
+    p.G = (int)G;
+    p.N = N;
+    p.m = (int)m;
+    return QKR_OK;
+}
+
+qkr_status vit_mrope_setup(void *stream, const float *inv_t, const float *inv_h,
+                           const float *inv_w, int64_t half_t, int64_t half_h, int64_t half_w,
+                           const int32_t *cu_seqlens, const int32_t *grids, int64_t G, int64_t N,
+                           int64_t spatial_merge, float *cos_out, float *sin_out)
+{
+    qkr::VitParams p = {};
+    qkr_status st = vit_common(cu_seqlens, grids, G, N, spatial_merge, p);
+    if (st != QKR_OK)
+        return st;
+    if (half_t < 0 || half_h < 0 || half_w < 0 || half_t + half_h + half_w < 1 ||
+        half_t + half_h + half_w > 4096)
+        return fail(QKR_ERR_INVALID_ARG, "per-axis lengths must be >= 0 and sum to [1, 4096]");
+    if ((half_t && !inv_t) || (half_h && !inv_h) || (half_w && !inv_w))
+        return fail(QKR_ERR_INVALID_ARG, "inv_freq of a non-empty axis is NULL");
+    if (N > 0 && (!cos_out || !sin_out))
+        return fail(QKR_ERR_INVALID_ARG, "cos_out and sin_out must be non-NULL");
+    if (!aligned4(cos_out) || !aligned4(sin_out) || !aligned4(inv_t) || !aligned4(inv_h) ||
+        !aligned4(inv_w))
+        return fail(QKR_ERR_UNSUPPORTED, "fp32 buffers must be 4-byte aligned");
+    p.inv[0] = inv_t;
+    p.inv[1] = inv_h;
+    p.inv[2] = inv_w;
+    p.half[0] = (int)half_t;
+    p.half[1] = (int)half_h;
+    p.half[2] = (int)half_w;
+    p.P = (int)(half_t + half_h + half_w);
+    p.cos_out = cos_out;
+    p.sin_out = sin_out;
+    if (N == 0) {
+        g_last = qkr::LaunchRecord();
+        g_error.clear();
+        return QKR_OK;
+    }
+    qkr::LaunchRecord rec;
+    qkr_status r = cuda_result(qkr::launch_vit_setup(p, static_cast<cudaStream_t>(stream), &rec),
+                               "vit setup launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
+}
+
+qkr_status rms_norm_residual(void *stream, const void *x, void *residual, const void *gamma,
+                             void *out, int64_t R, int64_t hidden, int64_t x_stride,
+                             int64_t res_stride, int64_t out_stride, float eps)
+{
+    if (R < 0)
+        return fail(QKR_ERR_INVALID_ARG, "R must be >= 0");
+    if (hidden < 8 || hidden > 65536 || hidden % 8)
+        return fail(QKR_ERR_UNSUPPORTED, "hidden %lld: need a multiple of 8 in [8, 65536]",
+                    (long long)hidden);
+    if (!(eps >= 0.f) || eps > 1.f)
+        return fail(QKR_ERR_INVALID_ARG, "eps must be finite and in [0, 1]");
+    if (R == 0) {
+        g_last = qkr::LaunchRecord();
+        g_error.clear();
+        return QKR_OK;
+    }
+    if (R > ((int64_t)1 << 31) - 1)
+        return fail(QKR_ERR_INVALID_ARG, "too many rows");
+    if (!x || !residual || !gamma || !out)
+        return fail(QKR_ERR_INVALID_ARG, "x, residual, gamma and out must be non-NULL");
+    if (!aligned16(x) || !aligned16(residual) || !aligned16(gamma) || !aligned16(out))
+        return fail(QKR_ERR_UNSUPPORTED, "pointers must be 16-byte aligned");
+    if (x_stride < hidden || res_stride < hidden || out_stride < hidden || x_stride % 8 ||
+        res_stride % 8 || out_stride % 8)
+        return fail(QKR_ERR_UNSUPPORTED,
+                    "row strides must be >= hidden and multiples of 8 elements");
+    if (!view_fits(R, x_stride, 1, 0, hidden) || !view_fits(R, res_stride, 1, 0, hidden) ||
+        !view_fits(R, out_stride, 1, 0, hidden))
+        return fail(QKR_ERR_INVALID_ARG, "view exceeds the address range");
+    const Span sx = view_span(x, R, x_stride, 1, 0, hidden);
+    const Span sr = view_span(residual, R, res_stride, 1, 0, hidden);
+    const Span so = view_span(out, R, out_stride, 1, 0, hidden);
+    if (overlap(sr, so) || overlap(sr, sx))
+        return fail(QKR_ERR_UNSUPPORTED, "residual must not overlap x or out");
+    if (overlap(sx, so) && !(x == out && x_stride == out_stride))
+        return fail(QKR_ERR_UNSUPPORTED, "out may only alias x exactly (same stride)");
+    qkr::RmsParams p;
+    p.x = static_cast<const __nv_bfloat16 *>(x);
+    p.res = static_cast<__nv_bfloat16 *>(residual);
+    p.gamma = static_cast<const __nv_bfloat16 *>(gamma);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.R = R;
+    p.hidden = (int)hidden;
+    p.xs = x_stride;
+    p.rs = res_stride;
+    p.os = out_stride;
+    p.eps = eps;
+    p.inv_hidden = 1.0f / (float)hidden;
+    qkr::LaunchRecord rec;
+    qkr_status r = cuda_result(
+        qkr::launch_rms_norm_residual(p, static_cast<cudaStream_t>(stream), &rec),
+        "rms norm launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
+}
+
+qkr_status qkr_section_map(void *stream, int32_t section_mode, const int32_t *sections,
+                           int64_t P, int8_t *axis_out)
+{
+    if (P < 1 || P > 4096)
+        return fail(QKR_ERR_INVALID_ARG, "P must be in [1, 4096]");
+    if (!axis_out)
+        return fail(QKR_ERR_INVALID_ARG, "axis_out is NULL");
+    int sec[4];
+    qkr_status st = check_sections(section_mode, sections, P, sec);
+    if (st != QKR_OK)
+        return st;
+    qkr::LaunchRecord rec;
+    qkr_status r = cuda_result(qkr::launch_section_map(section_mode, sec, (int)P, axis_out,
+                                                       static_cast<cudaStream_t>(stream), &rec),
+                               "section map launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
+}
+
+qkr_status qkr_vit_positions(void *stream, const int32_t *cu_seqlens, const int32_t *grids,
+                             int64_t G, int64_t N, int64_t spatial_merge, int32_t *pos_out)
+{
+    qkr::VitParams p = {};
+    qkr_status st = vit_common(cu_seqlens, grids, G, N, spatial_merge, p);
+    if (st != QKR_OK)
+        return st;
+    if (N > 0 && (!pos_out || !aligned4(pos_out)))
+        return fail(QKR_ERR_INVALID_ARG, "pos_out must be a non-NULL 4-byte aligned pointer");
+    if (N == 0) {
+        g_last = qkr::LaunchRecord();
+        g_error.clear();
+        return QKR_OK;
+    }
+    qkr::LaunchRecord rec;
+    qkr_status r = cuda_result(
+        qkr::launch_vit_positions(p, pos_out, static_cast<cudaStream_t>(stream), &rec),
+        "vit positions launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
+}
+
+}  // extern "C"

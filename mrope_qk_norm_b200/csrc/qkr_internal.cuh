@@ -1,0 +1,160 @@
+// qkr_internal.cuh -- device helpers and launch descriptors shared by the
+// CUDA translation units of the library (not part of the public ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qkr.h"
+
+namespace qkr {
+
+// ---------------------------------------------------------------- bf16 x8 --
+// A 16-byte vector holds 8 consecutive bf16 elements; element 2i sits in the
+// low half of word i.
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8])
+{
+    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]),
+                      pack2(f[6], f[7]));
+}
+
+__device__ __forceinline__ float round_bf16(float x)
+{
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// Streaming (evict-first) 16-byte global accesses for data touched once.
+__device__ __forceinline__ uint4 ld_stream(const void *p)
+{
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void st_stream(void *p, const uint4 &v)
+{
+    __stcs(reinterpret_cast<uint4 *>(p), v);
+}
+// Cached read-only 16-byte load for data every row reuses (gamma).
+__device__ __forceinline__ uint4 ld_reuse(const void *p)
+{
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// ------------------------------------------------------------ section rule --
+// Axis (0 t, 1 h, 2 w, 3 e) of rotated pair j under a section mode; the
+// rules are stated in include/qkr.h next to QKR_SECTIONS_*.
+__device__ __forceinline__ int section_axis(int mode, const int (&sec)[4], int j)
+{
+    if (mode == QKR_SECTIONS_NONE)
+        return 0;
+    const int st = sec[0], sh = sec[1], sw = sec[2];
+    if (mode == QKR_SECTIONS_IMROPE) {
+        const int sector = j % (st + sh + sw + sec[3]);
+        const int cls = sector % 3;                       // 0 t, 1 h, 2 w
+        const int quota = cls == 0 ? st : (cls == 1 ? sh : sw);
+        return sector < 3 * quota ? cls : 3;
+    }
+    const int m = min(st, min(sh, sw));
+    if (mode != QKR_SECTIONS_CONTIGUOUS && j < 3 * m)
+        return j % 3;
+    if (mode == QKR_SECTIONS_INTERLEAVED_QUOTA) {
+        int k = j - 3 * m;
+        if (k < st - m)
+            return 0;
+        k -= st - m;
+        return k < sh - m ? 1 : 2;
+    }
+    return j < st ? 0 : (j < st + sh ? 1 : 2);
+}
+
+// ---------------------------------------------------- rope row descriptors --
+
+struct RopeStreamDev {
+    const __nv_bfloat16 *q;   // already advanced by the storage offset
+    const __nv_bfloat16 *k;
+    int64_t q_ts, q_hs, k_ts, k_hs;
+    const __nv_bfloat16 *gq;
+    const __nv_bfloat16 *gk;
+};
+
+struct RopeParams {
+    RopeStreamDev st[2];
+    int64_t split;            // joint row where stream 1 starts (INT64_MAX: one stream)
+    __nv_bfloat16 *q_out;
+    __nv_bfloat16 *k_out;
+    int64_t qo_ts, ko_ts;
+    int64_t T;                // joint tokens in this launch
+    int Hq, Hk, D, rot, P;
+    int rows_per_token;       // Hq + Hk
+    int tokens_per_cta;
+    float eps, inv_D;
+    int norm, round_norm;
+    int angle_kind, section_mode;
+    int sec[4];
+    const int32_t *pos;
+    int64_t pos_rs;
+    const float *inv_freq;
+    const float *cos;
+    const float *sin;
+    int64_t ld, plane_stride;
+    int64_t token_offset;
+};
+
+struct LaunchRecord {
+    int kernel = QKR_KERNEL_NONE;
+    int lanes_per_row = 0, slots = 0, tokens_per_cta = 0, cluster = 1, block = 0;
+    int64_t grid = 0, launches = 0;
+};
+
+// Each launcher enqueues exactly one kernel and returns the CUDA launch status.
+cudaError_t launch_rope_rows(const RopeParams &p, int pairing, cudaStream_t stream,
+                             LaunchRecord *rec);
+
+struct VitParams {
+    const float *inv[3];
+    int half[3];
+    int P;
+    const int32_t *cu;
+    const int32_t *grids;
+    int G;
+    int64_t N;
+    int m;
+    float *cos_out;
+    float *sin_out;
+};
+cudaError_t launch_vit_setup(const VitParams &p, cudaStream_t stream, LaunchRecord *rec);
+cudaError_t launch_vit_positions(const VitParams &p, int32_t *pos_out, cudaStream_t stream,
+                                 LaunchRecord *rec);
+cudaError_t launch_section_map(int mode, const int (&sec)[4], int P, int8_t *out,
+                               cudaStream_t stream, LaunchRecord *rec);
+
+struct RmsParams {
+    const __nv_bfloat16 *x;
+    __nv_bfloat16 *res;
+    const __nv_bfloat16 *gamma;
+    __nv_bfloat16 *out;
+    int64_t R;
+    int hidden;
+    int64_t xs, rs, os;
+    float eps, inv_hidden;
+};
+cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream,
+                                     LaunchRecord *rec);
+
+}  // namespace qkr

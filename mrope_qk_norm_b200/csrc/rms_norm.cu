@@ -1,0 +1,259 @@
+// rms_norm.cu -- hidden-size RMSNorm with fused residual add.
+//
+// s = bf16(x + residual) is written back to residual; out = s * rsqrt(mean(s^2)
+// + eps) * gamma with an fp32 sum of squares of the bf16-rounded s (vllm.cpp
+// #185: the residual stream carries bf16 rounding; vLLM #26234: vectorised
+// reads of the row for the variance).
+//
+// B200 mapping.  Each thread keeps VPT 16-byte vectors of the row in
+// registers, so the row crosses HBM exactly once (read x and residual, write
+// residual and out).  The occupancy problem of vllm.cpp #185 (one workgroup
+// per row leaves the GPU idle when a decode step has one row) is solved with
+// a thread-block cluster: when rows are too few to fill the 148 SMs, each row
+// is split across a cluster of up to 16 CTAs, every CTA reduces its slice,
+// the partial sums are exchanged through distributed shared memory (read by
+// every CTA in rank order, so all CTAs get the same bit-identical total), and
+// each CTA normalises its slice.  No global scratch, no atomics, no spin-wait
+// on a flag: the cluster barrier's co-residency is guaranteed by the hardware.
+
+#include <cooperative_groups.h>
+
+#include <climits>
+
+#include "qkr_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace qkr {
+namespace {
+
+constexpr int kMaxThreads = 1024;
+
+// Sum over the block, identical in every thread; fixed order.
+__device__ __forceinline__ float block_sum(float v, float *red)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = (blockDim.x + 31) >> 5;
+    if (lane == 0)
+        red[warp] = v;
+    __syncthreads();
+    float t = 0.f;
+    for (int w = 0; w < nwarps; ++w)
+        t += red[w];
+    return t;
+}
+
+// Loads the slice [v0, v1) of a row (vector units), forms s = bf16(x + res),
+// writes it back to residual and returns the fp32 sum of s^2 of this thread.
+template <int VPT>
+__device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v0, int v1,
+                                          float (&s)[VPT][8], bool (&live)[VPT])
+{
+    const __nv_bfloat16 *xr = p.x + row * p.xs;
+    __nv_bfloat16 *rr = p.res + row * p.rs;
+    uint4 xv[VPT], rv[VPT];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int v = v0 + threadIdx.x + k * blockDim.x;
+        live[k] = v < v1;
+        if (live[k]) {
+            xv[k] = ld_stream(xr + 8 * v);
+            rv[k] = ld_stream(rr + 8 * v);
+        } else {
+            xv[k] = make_uint4(0, 0, 0, 0);
+            rv[k] = xv[k];
+        }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        float a[8], b[8];
+        unpack8(xv[k], a);
+        unpack8(rv[k], b);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            s[k][e] = a[e] + b[e];
+        const uint4 packed = pack8(s[k]);
+        unpack8(packed, s[k]);  // the residual stream is bf16: normalise the rounded sum
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            ss = fmaf(s[k][e], s[k][e], ss);
+        if (live[k])
+            st_stream(rr + 8 * (v0 + threadIdx.x + k * blockDim.x), packed);
+    }
+    return ss;
+}
+
+template <int VPT>
+__device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int v0,
+                                            float inv_rms, float (&s)[VPT][8],
+                                            const bool (&live)[VPT])
+{
+    __nv_bfloat16 *orow = p.out + row * p.os;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        if (!live[k])
+            continue;
+        const int v = v0 + threadIdx.x + k * blockDim.x;
+        float g[8];
+        unpack8(ld_reuse(p.gamma + 8 * v), g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            s[k][e] = (s[k][e] * inv_rms) * g[e];
+        st_stream(orow + 8 * v, pack8(s[k]));
+    }
+}
+
+// One CTA per row.
+template <int VPT>
+__global__ void __launch_bounds__(kMaxThreads) rms_rows_kernel(const __grid_constant__ RmsParams p)
+{
+    __shared__ float red[32];
+    const int64_t row = blockIdx.x;
+    float s[VPT][8];
+    bool live[VPT];
+    const float ss = load_sum<VPT>(p, row, 0, p.hidden >> 3, s, live);
+    const float total = block_sum(ss, red);
+    const float inv_rms = rsqrtf(fmaf(total, p.inv_hidden, p.eps));
+    scale_store<VPT>(p, row, 0, inv_rms, s, live);
+}
+
+// One cluster per row; CTA `rank` owns vectors [rank*per, (rank+1)*per).
+template <int VPT>
+__global__ void __launch_bounds__(kMaxThreads)
+rms_cluster_kernel(const __grid_constant__ RmsParams p)
+{
+    __shared__ float red[32];
+    __shared__ float partial;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int cs = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    const int64_t row = blockIdx.x / cs;
+    const int nvec = p.hidden >> 3;
+    const int per = (nvec + cs - 1) / cs;
+    const int v0 = rank * per;
+    const int v1 = min(v0 + per, nvec);
+
+    float s[VPT][8];
+    bool live[VPT];
+    const float ss = load_sum<VPT>(p, row, v0, v1, s, live);
+    const float mine = block_sum(ss, red);
+    if (threadIdx.x == 0)
+        partial = mine;
+    cluster.sync();  // every CTA's partial is visible cluster-wide
+    float total = 0.f;
+    for (int r = 0; r < cs; ++r)
+        total += *cluster.map_shared_rank(&partial, r);
+    cluster.barrier_arrive();  // done reading the other CTAs' shared memory
+    const float inv_rms = rsqrtf(fmaf(total, p.inv_hidden, p.eps));
+    scale_store<VPT>(p, row, v0, inv_rms, s, live);
+    cluster.barrier_wait();    // no CTA leaves while its partial may still be read
+}
+
+using Fn = void (*)(RmsParams);
+
+Fn rows_fn(int vpt)
+{
+    switch (vpt) {
+    case 1: return rms_rows_kernel<1>;
+    case 2: return rms_rows_kernel<2>;
+    case 4: return rms_rows_kernel<4>;
+    case 8: return rms_rows_kernel<8>;
+    default: return nullptr;
+    }
+}
+
+Fn cluster_fn(int vpt)
+{
+    switch (vpt) {
+    case 1: return rms_cluster_kernel<1>;
+    case 2: return rms_cluster_kernel<2>;
+    case 4: return rms_cluster_kernel<4>;
+    case 8: return rms_cluster_kernel<8>;
+    default: return nullptr;
+    }
+}
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+// Smallest power-of-two vectors-per-thread keeping the block at or under
+// `target` threads (and never above 1024).
+void shape(int vectors, int target, int &vpt, int &threads)
+{
+    vpt = 1;
+    while (vpt < 8 && (vectors + vpt - 1) / vpt > target)
+        vpt <<= 1;
+    threads = (vectors + vpt - 1) / vpt;
+    threads = ((threads + 31) / 32) * 32;
+    if (threads > kMaxThreads)
+        threads = kMaxThreads;
+}
+
+}  // namespace
+
+cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, LaunchRecord *rec)
+{
+    const int nvec = p.hidden >> 3;
+    const int target_ctas = 2 * sm_count();
+    int cs = 1;
+    if (p.R < target_ctas) {
+        while (cs < 16 && p.R * cs < target_ctas && nvec / (2 * cs) >= 32)
+            cs <<= 1;
+    }
+    int vpt, threads;
+    const int per = (nvec + cs - 1) / cs;
+    shape(per, 256, vpt, threads);
+    if ((int64_t)threads * vpt < per)
+        return cudaErrorInvalidConfiguration;
+    const int64_t grid = p.R * cs;
+    if (grid > INT_MAX)
+        return cudaErrorInvalidConfiguration;
+
+    cudaError_t err;
+    if (cs == 1) {
+        rows_fn(vpt)<<<(unsigned)grid, threads, 0, stream>>>(p);
+        err = cudaGetLastError();
+    } else {
+        Fn fn = cluster_fn(vpt);
+        if (cs > 8) {
+            err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (err != cudaSuccess)
+                return err;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, fn, p);
+    }
+    if (err == cudaSuccess && rec) {
+        *rec = LaunchRecord();
+        rec->kernel = cs == 1 ? QKR_KERNEL_RMS_ROWS : QKR_KERNEL_RMS_CLUSTER;
+        rec->slots = vpt;
+        rec->cluster = cs;
+        rec->block = threads;
+        rec->grid = grid;
+        rec->launches = 1;
+    }
+    return err;
+}
+
+}  // namespace qkr

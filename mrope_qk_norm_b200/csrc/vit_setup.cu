@@ -1,0 +1,168 @@
+// vit_setup.cu -- ViT mRoPE cos/sin plane setup (vLLM mrope_vit_setup page:
+// VitMropeSetup and _vit_mrope_setup_kernel) plus the two debug kernels that
+// expose the section rule and the grid-to-position mapping to the tests.
+//
+// B200 mapping.  The setup writes 2 * 4 bytes per (token, section column),
+// computing one sincosf per cell; it is store-bound at large N and
+// launch-bound at small N.  A CTA covers kTokens tokens: one thread per token
+// derives (t, h, w) once into shared memory, then all threads walk the
+// tokens' (token, column) cells with consecutive threads on consecutive
+// columns, so each warp's stores fall into a few contiguous runs of a plane.
+
+#include <climits>
+
+#include "qkr_internal.cuh"
+
+namespace qkr {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTokens = 32;
+
+// (t, h, w) of token n.  The grid is the g with cu[g] <= n < cu[g+1]
+// (binary search over the nondecreasing boundaries; empty grids are never
+// selected).  Inside a frame of h*w tokens, tokens come in m x m merge blocks
+// in row-major block order, each block's patches in row-major order.
+__device__ __forceinline__ void token_position(const int32_t *cu, const int32_t *grids, int G,
+                                               int64_t n, int m, int &tp, int &hp, int &wp)
+{
+    int lo = 0, hi = G;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)__ldg(cu + mid + 1) <= n)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    const int g = lo < G ? lo : G - 1;
+    const int64_t local = n - (int64_t)__ldg(cu + g);
+    const int h = __ldg(grids + 3 * g + 1);
+    const int w = __ldg(grids + 3 * g + 2);
+    const int64_t frame = max((int64_t)h * w, (int64_t)1);
+    tp = (int)(local / frame);
+    const int64_t in_frame = local - (int64_t)tp * frame;
+    const int mm = m * m;
+    const int64_t block = in_frame / mm;        // merge-block index in the frame
+    const int patch = (int)(in_frame - block * mm);
+    const int64_t blocks_per_row = max(w / m, 1);
+    const int64_t brow = block / blocks_per_row;
+    const int64_t bcol = block - brow * blocks_per_row;
+    hp = (int)(brow * m + patch / m);
+    wp = (int)(bcol * m + patch % m);
+}
+
+__global__ void __launch_bounds__(kThreads) vit_setup_kernel(const __grid_constant__ VitParams p)
+{
+    __shared__ int spos[3][kTokens];
+    const int64_t n0 = (int64_t)blockIdx.x * kTokens;
+    const int ntok = (int)min((int64_t)kTokens, p.N - n0);
+    if (threadIdx.x < ntok) {
+        int tp, hp, wp;
+        token_position(p.cu, p.grids, p.G, n0 + threadIdx.x, p.m, tp, hp, wp);
+        spos[0][threadIdx.x] = tp;
+        spos[1][threadIdx.x] = hp;
+        spos[2][threadIdx.x] = wp;
+    }
+    __syncthreads();
+
+    const int P = p.P;
+    const int end_t = p.half[0], end_h = p.half[0] + p.half[1];
+    for (int idx = threadIdx.x; idx < ntok * P; idx += kThreads) {
+        const int tt = idx / P;
+        const int col = idx - tt * P;
+        const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
+        const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
+        const float theta = __fmul_rn((float)spos[axis][tt], __ldg(p.inv[axis] + (col - off)));
+        float s, c;
+        sincosf(theta, &s, &c);
+        const int64_t at = ((int64_t)axis * p.N + n0 + tt) * P + col;
+        p.cos_out[at] = c;
+        p.sin_out[at] = s;
+    }
+}
+
+__global__ void vit_positions_kernel(const __grid_constant__ VitParams p, int32_t *out)
+{
+    const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= p.N)
+        return;
+    int tp, hp, wp;
+    token_position(p.cu, p.grids, p.G, n, p.m, tp, hp, wp);
+    out[n] = tp;
+    out[p.N + n] = hp;
+    out[2 * p.N + n] = wp;
+}
+
+struct SectionArgs {
+    int mode;
+    int sec[4];
+    int P;
+};
+
+__global__ void section_map_kernel(const __grid_constant__ SectionArgs a, int8_t *out)
+{
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j < a.P)
+        out[j] = (int8_t)section_axis(a.mode, a.sec, j);
+}
+
+}  // namespace
+
+cudaError_t launch_vit_setup(const VitParams &p, cudaStream_t stream, LaunchRecord *rec)
+{
+    const int64_t grid = (p.N + kTokens - 1) / kTokens;
+    if (grid > INT_MAX)
+        return cudaErrorInvalidConfiguration;
+    vit_setup_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(p);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess && rec) {
+        *rec = LaunchRecord();
+        rec->kernel = QKR_KERNEL_VIT_SETUP;
+        rec->tokens_per_cta = kTokens;
+        rec->block = kThreads;
+        rec->grid = grid;
+        rec->launches = 1;
+    }
+    return err;
+}
+
+cudaError_t launch_vit_positions(const VitParams &p, int32_t *pos_out, cudaStream_t stream,
+                                 LaunchRecord *rec)
+{
+    const int64_t grid = (p.N + kThreads - 1) / kThreads;
+    if (grid > INT_MAX)
+        return cudaErrorInvalidConfiguration;
+    vit_positions_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(p, pos_out);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess && rec) {
+        *rec = LaunchRecord();
+        rec->kernel = QKR_KERNEL_VIT_POSITIONS;
+        rec->block = kThreads;
+        rec->grid = grid;
+        rec->launches = 1;
+    }
+    return err;
+}
+
+cudaError_t launch_section_map(int mode, const int (&sec)[4], int P, int8_t *out,
+                               cudaStream_t stream, LaunchRecord *rec)
+{
+    SectionArgs a;
+    a.mode = mode;
+    for (int i = 0; i < 4; ++i)
+        a.sec[i] = sec[i];
+    a.P = P;
+    const int grid = (P + 127) / 128;
+    section_map_kernel<<<grid, 128, 0, stream>>>(a, out);
+    cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess && rec) {
+        *rec = LaunchRecord();
+        rec->kernel = QKR_KERNEL_SECTION_MAP;
+        rec->block = 128;
+        rec->grid = grid;
+        rec->launches = 1;
+    }
+    return err;
+}
+
+}  // namespace qkr

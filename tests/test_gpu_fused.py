@@ -1,0 +1,210 @@
+"""GPU parity of fused_qk_norm_rope against the CPU oracle.
+
+Covers the single-stream configuration (T=16, H=4, D=64, NeoX, positions
+0..15, seed 0), the joint text/image configuration at full size (512 + 4096
+tokens, 24 heads, D=128, fp32 [4608, 64] cos/sin table, both pairings), the
+2^31-element storage-offset variant on either stream, strided views, the
+bf16-rounded-normalised-value contract, every kernel layout and ragged
+shapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mrope_qk_norm_b200 as qkr
+import oracle
+import workloads as W
+from tests._gpu_util import Guarded, assert_bf16_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _angle_desc(angle, dev_keep):
+    if angle.kind == W.ANGLE_POSITIONS:
+        pos = to_dev(torch.as_tensor(np.asarray(angle.positions), dtype=torch.int32))
+        inv = to_dev(torch.as_tensor(np.asarray(angle.inv_freq), dtype=torch.float32))
+        dev_keep += [pos, inv]
+        return qkr.angle_positions(pos, inv, angle.section_mode, angle.sections, angle.token_offset)
+    cos = to_dev(torch.as_tensor(np.asarray(angle.cos), dtype=torch.float32))
+    sin = to_dev(torch.as_tensor(np.asarray(angle.sin), dtype=torch.float32))
+    dev_keep += [cos, sin]
+    return qkr.angle_table(cos, sin, angle.section_mode, angle.sections, angle.token_offset)
+
+
+def run_fused(w: W.RopeWorkload, flags=0, guard=True):
+    keep = []
+    streams = []
+    for s in w.streams:
+        q, k, gq, gk = (to_dev(s.q), to_dev(s.k), to_dev(s.gamma_q), to_dev(s.gamma_k))
+        keep += [q, k, gq, gk]
+        streams.append((q, k, gq, gk))
+    T = w.n_tokens
+    qo = Guarded((T, w.Hq, w.D))
+    ko = Guarded((T, w.Hk, w.D))
+    a = _angle_desc(w.angle, keep)
+    qkr.fused_qk_norm_rope(streams, qo.tensor, ko.tensor, w.rot, w.pairing, w.eps, a, flags)
+    torch.cuda.synchronize()
+    qo.check()
+    ko.check()
+    return qo.tensor, ko.tensor
+
+
+def check_against_oracle(w, flags=0, what=""):
+    q, k = run_fused(w, flags)
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle,
+                                 norm=w.norm, round_normalized=bool(flags & 1))
+    sq = assert_bf16_close(q, rq, what + " q")
+    sk = assert_bf16_close(k, rk, what + " k")
+    return q, k, sq, sk
+
+
+@pytest.mark.parametrize("pairing", [W.PAIRING_NEOX, W.PAIRING_GPTJ])
+def test_single_stream_config(pairing):
+    w = W.config1(pairing=pairing)
+    check_against_oracle(w, what="config1")
+    info = qkr.last_launch()
+    assert info["kernel_name"] == ("rope_paired" if pairing == W.PAIRING_NEOX else "rope_vector")
+    assert info["launches"] == 1
+
+
+@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
+def test_joint_config_full_size(pairing):
+    w = W.config3(pairing=pairing)
+    q, k, _, _ = check_against_oracle(w, what="joint")
+    # the joint launch equals the two streams launched separately, bit for bit
+    txt = W.RopeWorkload("txt", w.streams[:1], w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    img_angle = W.AngleInputs(kind=W.ANGLE_TABLE, cos=w.angle.cos, sin=w.angle.sin,
+                              token_offset=w.streams[0].q.shape[0])
+    img = W.RopeWorkload("img", w.streams[1:], w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, img_angle)
+    qt, kt = run_fused(txt)
+    qi, ki = run_fused(img)
+    assert torch.equal(q.view(torch.int16), torch.cat([qt, qi]).view(torch.int16))
+    assert torch.equal(k.view(torch.int16), torch.cat([kt, ki]).view(torch.int16))
+
+
+def test_joint_small_ragged_vs_oracle():
+    # 37 text + 5x7 image tokens: several CTA tiles and a ragged last tile
+    for pairing in (W.PAIRING_GPTJ, W.PAIRING_NEOX):
+        w = W.config3(seed=13, T_txt=37, img_h=5, img_w=7, H=6, D=128, pairing=pairing)
+        check_against_oracle(w, what="joint small")
+
+
+@pytest.mark.parametrize("which", [0, 1])
+@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
+def test_large_storage_offset(which, pairing):
+    """One stream lives 2^31 elements into its storage (needs > 8 GiB free)."""
+    free, _ = torch.cuda.mem_get_info()
+    if free < 12 * 2 ** 30:
+        pytest.skip("needs 12 GiB of free device memory")
+    w = W.config3(seed=17, T_txt=64, img_h=16, img_w=16, H=24, D=128, pairing=pairing)
+    ref_q, ref_k = run_fused(w)
+    keep, streams = [], []
+    off = 2 ** 31
+    for i, s in enumerate(w.streams):
+        q, k = to_dev(s.q), to_dev(s.k)
+        if i == which:
+            big_q = torch.empty(off + q.numel(), dtype=torch.bfloat16, device="cuda")
+            big_q[off:].copy_(q.reshape(-1))
+            big_k = torch.empty(off + k.numel(), dtype=torch.bfloat16, device="cuda")
+            big_k[off:].copy_(k.reshape(-1))
+            q = big_q[off:].view(q.shape)
+            k = big_k[off:].view(k.shape)
+            assert q.storage_offset() == off
+            keep += [big_q, big_k]
+        gq, gk = to_dev(s.gamma_q), to_dev(s.gamma_k)
+        keep += [q, k, gq, gk]
+        streams.append((q, k, gq, gk))
+    T = w.n_tokens
+    qo = torch.empty(T, w.Hq, w.D, dtype=torch.bfloat16, device="cuda")
+    ko = torch.empty(T, w.Hk, w.D, dtype=torch.bfloat16, device="cuda")
+    a = _angle_desc(w.angle, keep)
+    qkr.fused_qk_norm_rope(streams, qo, ko, w.rot, w.pairing, w.eps, a)
+    torch.cuda.synchronize()
+    assert torch.equal(qo.view(torch.int16), ref_q.view(torch.int16))
+    assert torch.equal(ko.view(torch.int16), ref_k.view(torch.int16))
+    del keep
+    torch.cuda.empty_cache()
+
+
+def test_strided_chunked_qkv_views():
+    # Q and K are views into a packed [T, 3, H, D] QKV buffer (zero-copy split).
+    g = torch.Generator().manual_seed(21)
+    T, H, D = 50, 8, 128
+    qkv = W.bf16_normal((T, 3, H, D), g)
+    gq = W.bf16_uniform((D,), 0.5, 1.5, g)
+    gk = W.bf16_uniform((D,), 0.5, 1.5, g)
+    inv = W.inv_freq(1e4, D // 2, D)
+    pos = torch.arange(3, 3 + T, dtype=torch.int32).view(1, T)
+    dq = to_dev(qkv)
+    dgq, dgk, dpos, dinv = to_dev(gq), to_dev(gk), to_dev(pos), to_dev(inv)
+    qo = torch.empty(T, H, D, dtype=torch.bfloat16, device="cuda")
+    ko = torch.empty_like(qo)
+    a = qkr.angle_positions(dpos, dinv)
+    qkr.fused_qk_norm_rope([(dq[:, 0], dq[:, 1], dgq, dgk)], qo, ko, D, W.PAIRING_NEOX, 1e-6, a)
+    torch.cuda.synchronize()
+    s = W.StreamInputs(qkv[:, 0].contiguous(), qkv[:, 1].contiguous(), gq, gk)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=inv)
+    rq, rk = oracle.qk_norm_rope([s], H, H, D, D, W.PAIRING_NEOX, 1e-6, A)
+    assert_bf16_close(qo, rq, "strided q")
+    assert_bf16_close(ko, rk, "strided k")
+
+
+@pytest.mark.parametrize("D,rot,pairing,kernel", [
+    (64, 64, W.PAIRING_NEOX, "rope_paired"),
+    (128, 128, W.PAIRING_NEOX, "rope_paired"),
+    (80, 64, W.PAIRING_NEOX, "rope_paired"),
+    (128, 64, W.PAIRING_NEOX, "rope_paired"),
+    (256, 256, W.PAIRING_NEOX, "rope_paired"),
+    (256, 96, W.PAIRING_NEOX, "rope_exchange"),
+    (96, 96, W.PAIRING_NEOX, "rope_paired"),
+    (32, 16, W.PAIRING_NEOX, "rope_paired"),
+    (64, 20, W.PAIRING_NEOX, "rope_exchange"),
+    (24, 2, W.PAIRING_NEOX, "rope_exchange"),
+    (8, 8, W.PAIRING_NEOX, "rope_exchange"),
+    (256, 256, W.PAIRING_GPTJ, "rope_vector"),
+    (80, 64, W.PAIRING_GPTJ, "rope_vector"),
+    (64, 22, W.PAIRING_GPTJ, "rope_vector"),
+    (8, 6, W.PAIRING_GPTJ, "rope_vector"),
+    (128, 0, W.PAIRING_NEOX, "rope_vector"),
+])
+def test_geometries(D, rot, pairing, kernel):
+    T = 45  # ragged against every tokens-per-CTA choice
+    pos = np.random.default_rng(D * 1000 + rot).integers(0, 100000, T).astype(np.int32)
+    inv = W.inv_freq(1e4, max(rot // 2, 1), max(rot, 2)).numpy()
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos[None], inv_freq=inv)
+    w = W.random_rope_case(D + rot, [T], 5, 3, D, rot, pairing, A)
+    check_against_oracle(w, what="D=%d rot=%d" % (D, rot))
+    assert qkr.last_launch()["kernel_name"] == kernel
+
+
+def test_round_normalized_contract():
+    w = W.config3(seed=23, T_txt=40, img_h=8, img_w=8, H=8, D=128)
+    check_against_oracle(w, flags=qkr.FLAG_ROUND_NORMALIZED_BF16, what="round-normalised")
+
+
+def test_zero_positions_is_pure_norm_and_deterministic():
+    g = torch.Generator().manual_seed(29)
+    T, H, D = 33, 4, 128
+    pos = np.zeros((1, T), dtype=np.int32)
+    inv = W.inv_freq(1e4, 64, 128).numpy()
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=inv)
+    w = W.random_rope_case(29, [T], H, H, D, D, W.PAIRING_NEOX, A)
+    q1, k1 = run_fused(w)
+    q2, k2 = run_fused(w)
+    assert torch.equal(q1.view(torch.int16), q2.view(torch.int16))
+    w0 = W.random_rope_case(29, [T], H, H, D, 0, W.PAIRING_NEOX, A)
+    q0, k0 = run_fused(w0)
+    assert torch.equal(q1.view(torch.int16), q0.view(torch.int16))
+    assert torch.equal(k1.view(torch.int16), k0.view(torch.int16))
+
+
+def test_empty_streams():
+    # an empty text stream and an empty call
+    w = W.config3(seed=31, T_txt=0, img_h=4, img_w=4, H=2, D=64)
+    check_against_oracle(w, what="empty text stream")
+    keep = []
+    a = _angle_desc(w.angle, keep)
+    e = torch.empty(0, 2, 64, dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(64, dtype=torch.bfloat16, device="cuda")
+    qkr.fused_qk_norm_rope([(e, e, g, g)], e, e, 64, 0, 1e-6, a)
+    assert qkr.last_launch()["launches"] == 0
