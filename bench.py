@@ -76,7 +76,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device: torch.device, period_s: float = 0.005):
         self.samples = []
         self.ok = False
         self.period = period_s
@@ -84,7 +84,9 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            # NVML ignores CUDA_VISIBLE_DEVICES: find the device by its UUID
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -290,19 +292,31 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20):
 
 # ------------------------------------------------------------- CPU oracle --
 
-def cpu_baseline(budget_s: float = 12.0) -> dict:
-    """The oracle as it stands, single-threaded, on a bounded token sample."""
+N_IMG_SAMPLE = 512
+
+
+def _oracle_sample():
+    """Bounded sample of the headline workload: all 512 text tokens and the
+    first 512 image tokens (the table rows of those tokens are used as is)."""
     import oracle
     w = W.config3()
-    n_img = 512
     s_txt = w.streams[0]
-    s_img = W.StreamInputs(w.streams[1].q[:n_img], w.streams[1].k[:n_img],
+    s_img = W.StreamInputs(w.streams[1].q[:N_IMG_SAMPLE], w.streams[1].k[:N_IMG_SAMPLE],
                            w.streams[1].gamma_q, w.streams[1].gamma_k)
-    tokens = s_txt.q.shape[0] + n_img
+    tokens = s_txt.q.shape[0] + N_IMG_SAMPLE
+
+    def step():
+        oracle.qk_norm_rope([s_txt, s_img], 24, 24, 128, 128, w.pairing, w.eps, w.angle)
+    return step, tokens
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    """The oracle as it stands, single-threaded, on a bounded token sample."""
+    step, tokens = _oracle_sample()
     t0 = time.perf_counter()
     calls = 0
     while True:
-        oracle.qk_norm_rope([s_txt, s_img], 24, 24, 128, 128, w.pairing, w.eps, w.angle)
+        step()
         calls += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -311,7 +325,32 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
             "kind": "oracle",
             "sample": "%d calls x %d tokens (all 512 text + first %d image tokens of the "
                       "headline workload), fp64 C oracle, one thread, %.1f s"
-                      % (calls, tokens, n_img, dt)}
+                      % (calls, tokens, N_IMG_SAMPLE, dt)}
+
+
+def reference_arm(args) -> dict:
+    """The CPU oracle timed like our arm: W untimed steps, then K timed steps,
+    each step one oracle call on the bounded sample."""
+    step, tokens = _oracle_sample()
+    for _ in range(min(args.warmup, 3)):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = round(args.steps * tokens / dt, 1)
+    sample = ("each step: one oracle call on %d tokens (all 512 text + first %d image tokens "
+              "of the headline workload), fp64 C oracle, one thread; %d steps in %.1f s"
+              % (tokens, N_IMG_SAMPLE, args.steps, dt))
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": min(args.warmup, 3),
+            "ms_per_step": round(1e3 * dt / max(args.steps, 1), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
 
 
 # ------------------------------------------------------------------- main --
@@ -325,6 +364,8 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the per-kernel rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--row-steps", type=int, default=200)
+    ap.add_argument("--row-warmup", type=int, default=20)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -335,15 +376,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = cpu_baseline(budget_s=max(2.0, min(60.0, 0.25 * max(args.steps, 1))))
-        line = {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": WORKLOAD, "sample": cb["sample"]},
-                "cpu_baseline": cb,
-                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
+        line = reference_arm(args)
         print(json.dumps(line))
         return 0
 
@@ -365,8 +398,7 @@ def main():
     sets = [FusedSet(w, dev) for _ in range(n_sets)]
     fns = [lambda s=s: s.launch(stream) for s in sets]
 
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else local)
+    sampler = ClockSampler(dev)
     sampler.start()
     for i in range(args.warmup):
         fns[i % n_sets]()
@@ -437,7 +469,7 @@ def main():
     if not args.no_rows:
         del sets, fns
         torch.cuda.empty_cache()
-        rows = measure_rows(dev, stream, peaks["hbm_gbs"])
+        rows = measure_rows(dev, stream, peaks["hbm_gbs"], args.row_steps, args.row_warmup)
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu:

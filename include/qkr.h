@@ -283,12 +283,19 @@ typedef struct qkr_launch_info {
     int32_t lanes_per_row;   /* rope kernels: lanes that share one head row */
     int32_t slots;           /* rope: 16-byte vectors per lane per row; rms: per thread */
     int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
+    int32_t heads_per_item;  /* rope: head rows a lane group loads together */
     int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
     int32_t block;           /* threads per CTA */
     int64_t grid;            /* CTAs launched */
     int64_t launches;        /* kernel launches enqueued (0 for an empty call) */
 } qkr_launch_info;
 qkr_status qkr_last_launch(qkr_launch_info *info);
+
+/* Launch-shape override for the rope kernels, for tuning sweeps: heads per
+ * work item (1..4) and tokens per CTA (1..16); 0 keeps the automatic choice.
+ * Process-wide; results are identical for every shape (each row's arithmetic
+ * does not depend on it).  Returns QKR_ERR_INVALID_ARG out of range. */
+qkr_status qkr_tune_rope_shape(int32_t heads_per_item, int32_t tokens_per_cta);
 
 /* Writes the axis (0 t, 1 h, 2 w, 3 e) of pairs 0..P-1 under a section mode
  * to axis_out (device int8 [P]) with the kernels' own section rule.

@@ -3,9 +3,9 @@
 Every function here takes torch tensors already on a CUDA device, checks
 their dtype/device, passes raw pointers, sizes and strides to the C ABI on
 the current torch stream, and raises ``QkrError`` on a non-zero status.  All
-arithmetic runs in the library's CUDA kernels; there is no CPU path.  If the
-shared library is missing the import fails: build it with
-``python -m mrope_qk_norm_b200.build``.
+arithmetic runs in the library's CUDA kernels; there is no CPU path.  The shared
+library is loaded on first use; if it is missing every call raises
+ImportError -- build it with ``python mrope_qk_norm_b200/build.py``.
 """
 from __future__ import annotations
 
@@ -29,7 +29,7 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
 
 EXPORTS = ("fused_qk_norm_rope", "mrope_apply", "vit_mrope_setup", "rms_norm_residual",
            "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
-           "qkr_vit_positions")
+           "qkr_vit_positions", "qkr_tune_rope_shape")
 
 
 class QkrError(RuntimeError):
@@ -60,6 +60,7 @@ class AngleDesc(ctypes.Structure):
 class LaunchInfo(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("lanes_per_row", ctypes.c_int32),
                 ("slots", ctypes.c_int32), ("tokens_per_cta", ctypes.c_int32),
+                ("heads_per_item", ctypes.c_int32),
                 ("cluster", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("grid", ctypes.c_int64), ("launches", ctypes.c_int64)]
 
@@ -81,6 +82,7 @@ def _load() -> ctypes.CDLL:
         "qkr_last_launch": [ctypes.POINTER(LaunchInfo)],
         "qkr_section_map": [V, I32, V, I64, V],
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
+        "qkr_tune_rope_shape": [I32, I32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -93,11 +95,23 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_lib_handle = None
 
 
 def lib() -> ctypes.CDLL:
-    return _lib
+    """The loaded libqkr.so (loaded on first use; raises if it is missing)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load()
+    return _lib_handle
+
+
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(lib(), name)
+
+
+_lib = _LazyLib()
 
 
 def version() -> str:
@@ -132,6 +146,11 @@ def _ptr_base(t, dtype, what):
     if t.dtype != dtype:
         raise ValueError("%s must be %s, got %s" % (what, dtype, t.dtype))
     return t.untyped_storage().data_ptr(), t.storage_offset()
+
+
+def tune_rope_shape(heads_per_item: int = 0, tokens_per_cta: int = 0) -> None:
+    """Override the rope kernels' launch shape (0 = automatic), for tuning."""
+    _check(_lib.qkr_tune_rope_shape(heads_per_item, tokens_per_cta))
 
 
 def last_launch() -> dict:

@@ -1,6 +1,6 @@
 """Build libqkr.so (sm_100a) in-tree with nvcc.
 
-    python -m mrope_qk_norm_b200.build [--ptxas-verbose]
+    python mrope_qk_norm_b200/build.py [--force] [--ptxas-verbose]
 
 Each .cu under csrc/ is compiled to an object in parallel, then linked into
 mrope_qk_norm_b200/libqkr.so with the CUDA runtime linked statically, so the

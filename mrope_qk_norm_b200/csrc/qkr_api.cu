@@ -332,10 +332,20 @@ qkr_status qkr_last_launch(qkr_launch_info *info)
     info->lanes_per_row = g_last.lanes_per_row;
     info->slots = g_last.slots;
     info->tokens_per_cta = g_last.tokens_per_cta;
+    info->heads_per_item = g_last.heads_per_item;
     info->cluster = g_last.cluster;
     info->block = g_last.block;
     info->grid = g_last.grid;
     info->launches = g_last.launches;
+    return QKR_OK;
+}
+
+qkr_status qkr_tune_rope_shape(int32_t heads_per_item, int32_t tokens_per_cta)
+{
+    if (heads_per_item < 0 || heads_per_item > 4 || tokens_per_cta < 0 || tokens_per_cta > 16)
+        return fail(QKR_ERR_INVALID_ARG, "heads_per_item in [0, 4], tokens_per_cta in [0, 16]");
+    qkr::set_rope_shape_override(heads_per_item, tokens_per_cta);
+    g_error.clear();
     return QKR_OK;
 }
 

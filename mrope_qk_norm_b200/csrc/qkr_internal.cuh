@@ -103,6 +103,8 @@ struct RopeParams {
     int Hq, Hk, D, rot, P;
     int rows_per_token;       // Hq + Hk
     int tokens_per_cta;
+    int pw;                   // (cos, sin) columns staged per token: P, or D/2 for GPT-J
+                              // (pairs in [P, D/2) get the identity (1, 0))
     float eps, inv_D;
     int norm, round_norm;
     int angle_kind, section_mode;
@@ -118,9 +120,13 @@ struct RopeParams {
 
 struct LaunchRecord {
     int kernel = QKR_KERNEL_NONE;
-    int lanes_per_row = 0, slots = 0, tokens_per_cta = 0, cluster = 1, block = 0;
+    int lanes_per_row = 0, slots = 0, tokens_per_cta = 0, heads_per_item = 0, cluster = 1,
+        block = 0;
     int64_t grid = 0, launches = 0;
 };
+
+// Launch-shape override of the rope kernels (0: automatic).
+void set_rope_shape_override(int heads_per_item, int tokens_per_cta);
 
 // Each launcher enqueues exactly one kernel and returns the CUDA launch status.
 cudaError_t launch_rope_rows(const RopeParams &p, int pairing, cudaStream_t stream,
