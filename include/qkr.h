@@ -284,6 +284,8 @@ typedef struct qkr_launch_info {
     int32_t slots;           /* rope: 16-byte vectors per lane per row; rms: per thread */
     int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
     int32_t heads_per_item;  /* rope: head rows a lane group loads together */
+    int32_t pipelined;       /* rope: 1 if rows were staged by bulk copies into a
+                                shared-memory ring (warp-specialised kernel) */
     int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
     int32_t block;           /* threads per CTA */
     int64_t grid;            /* CTAs launched */
@@ -291,11 +293,21 @@ typedef struct qkr_launch_info {
 } qkr_launch_info;
 qkr_status qkr_last_launch(qkr_launch_info *info);
 
-/* Launch-shape override for the rope kernels, for tuning sweeps: heads per
- * work item (1..4) and tokens per CTA (1..16); 0 keeps the automatic choice.
- * Process-wide; results are identical for every shape (each row's arithmetic
- * does not depend on it).  Returns QKR_ERR_INVALID_ARG out of range. */
-qkr_status qkr_tune_rope_shape(int32_t heads_per_item, int32_t tokens_per_cta);
+/* Launch-shape override for the rope kernels, for tuning sweeps.  pipeline:
+ * 0 automatic, 1 register kernel only, 2 bulk-copy pipelined kernel only
+ * (calls it cannot serve then fail with QKR_ERR_CUDA); heads per work item
+ * (1..8, register kernel) and tokens per CTA or per pipeline tile (1..32);
+ * 0 keeps the automatic choice.  Process-wide.  Every shape computes
+ * bit-identical results: a row's arithmetic does not depend on it.
+ * Returns QKR_ERR_INVALID_ARG out of range. */
+qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta);
+
+/* Device status word of the library on the current device (0 = healthy).
+ * Kernels that wait on shared-memory barriers give every wait a time budget;
+ * a wait that runs out sets a bit here (1: producer, 2: consumer) and the
+ * kernel returns early instead of hanging.  Synchronous (copies the word to
+ * the host); reset != 0 clears it.  Not for the hot path. */
+qkr_status qkr_device_status(uint32_t *status, int32_t reset);
 
 /* Writes the axis (0 t, 1 h, 2 w, 3 e) of pairs 0..P-1 under a section mode
  * to axis_out (device int8 [P]) with the kernels' own section rule.

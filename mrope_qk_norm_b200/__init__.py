@@ -29,7 +29,7 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
 
 EXPORTS = ("fused_qk_norm_rope", "mrope_apply", "vit_mrope_setup", "rms_norm_residual",
            "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
-           "qkr_vit_positions", "qkr_tune_rope_shape")
+           "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status")
 
 
 class QkrError(RuntimeError):
@@ -60,7 +60,7 @@ class AngleDesc(ctypes.Structure):
 class LaunchInfo(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("lanes_per_row", ctypes.c_int32),
                 ("slots", ctypes.c_int32), ("tokens_per_cta", ctypes.c_int32),
-                ("heads_per_item", ctypes.c_int32),
+                ("heads_per_item", ctypes.c_int32), ("pipelined", ctypes.c_int32),
                 ("cluster", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("grid", ctypes.c_int64), ("launches", ctypes.c_int64)]
 
@@ -82,7 +82,8 @@ def _load() -> ctypes.CDLL:
         "qkr_last_launch": [ctypes.POINTER(LaunchInfo)],
         "qkr_section_map": [V, I32, V, I64, V],
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
-        "qkr_tune_rope_shape": [I32, I32],
+        "qkr_tune_rope": [I32, I32, I32],
+        "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -148,9 +149,16 @@ def _ptr_base(t, dtype, what):
     return t.untyped_storage().data_ptr(), t.storage_offset()
 
 
-def tune_rope_shape(heads_per_item: int = 0, tokens_per_cta: int = 0) -> None:
+def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 0) -> None:
     """Override the rope kernels' launch shape (0 = automatic), for tuning."""
-    _check(_lib.qkr_tune_rope_shape(heads_per_item, tokens_per_cta))
+    _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta))
+
+
+def device_status(reset: bool = False) -> int:
+    """The library's device status word (0 = healthy); synchronous."""
+    v = ctypes.c_uint32(0)
+    _check(_lib.qkr_device_status(ctypes.byref(v), int(reset)))
+    return int(v.value)
 
 
 def last_launch() -> dict:
@@ -180,6 +188,7 @@ def stream_desc(q, k, gamma_q, gamma_k) -> StreamDesc:
     d.n_tokens = q.shape[0]
     d.gamma_q = _ptr(gamma_q, bf, "gamma_q")
     d.gamma_k = _ptr(gamma_k, bf, "gamma_k")
+    d._keep = (q, k, gamma_q, gamma_k)  # the descriptor holds raw pointers into these
     return d
 
 
@@ -198,6 +207,7 @@ def angle_positions(positions, inv_freq, section_mode=SECTIONS_NONE, sections=No
     a.pos_row_stride = positions.shape[-1]
     a.inv_freq = _ptr(inv_freq, torch.float32, "inv_freq")
     a.token_offset = token_offset
+    a._keep = (positions, inv_freq)  # the descriptor holds raw pointers into these
     return a
 
 
@@ -220,6 +230,7 @@ def angle_table(cos, sin, section_mode=SECTIONS_NONE, sections=None, token_offse
     a.ld = c3.stride(1)
     a.plane_stride = c3.stride(0) if c3.shape[0] > 1 else c3.shape[1] * c3.stride(1)
     a.token_offset = token_offset
+    a._keep = (c3, s3)  # the descriptor holds raw pointers into these
     return a
 
 

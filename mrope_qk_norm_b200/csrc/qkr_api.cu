@@ -333,6 +333,7 @@ qkr_status qkr_last_launch(qkr_launch_info *info)
     info->slots = g_last.slots;
     info->tokens_per_cta = g_last.tokens_per_cta;
     info->heads_per_item = g_last.heads_per_item;
+    info->pipelined = g_last.pipelined;
     info->cluster = g_last.cluster;
     info->block = g_last.block;
     info->grid = g_last.grid;
@@ -340,13 +341,25 @@ qkr_status qkr_last_launch(qkr_launch_info *info)
     return QKR_OK;
 }
 
-qkr_status qkr_tune_rope_shape(int32_t heads_per_item, int32_t tokens_per_cta)
+qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta)
 {
-    if (heads_per_item < 0 || heads_per_item > 4 || tokens_per_cta < 0 || tokens_per_cta > 16)
-        return fail(QKR_ERR_INVALID_ARG, "heads_per_item in [0, 4], tokens_per_cta in [0, 16]");
-    qkr::set_rope_shape_override(heads_per_item, tokens_per_cta);
+    if (pipeline < 0 || pipeline > 2 || heads_per_item < 0 || heads_per_item > 8 ||
+        tokens_per_cta < 0 || tokens_per_cta > 32)
+        return fail(QKR_ERR_INVALID_ARG,
+                    "pipeline in [0, 2], heads_per_item in [0, 8], tokens_per_cta in [0, 32]");
+    qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta);
     g_error.clear();
     return QKR_OK;
+}
+
+qkr_status qkr_device_status(uint32_t *status, int32_t reset)
+{
+    if (!status)
+        return fail(QKR_ERR_INVALID_ARG, "status is NULL");
+    unsigned v = 0;
+    qkr_status r = cuda_result(qkr::read_device_status(&v, reset != 0), "device status read");
+    *status = v;
+    return r;
 }
 
 qkr_status fused_qk_norm_rope(void *stream, const qkr_stream_desc *streams, int32_t n_streams,

@@ -103,6 +103,7 @@ struct RopeParams {
     int Hq, Hk, D, rot, P;
     int rows_per_token;       // Hq + Hk
     int tokens_per_cta;
+    int heads_per_item;       // heads of one token and kind a lane group processes together
     int pw;                   // (cos, sin) columns staged per token: P, or D/2 for GPT-J
                               // (pairs in [P, D/2) get the identity (1, 0))
     float eps, inv_D;
@@ -121,12 +122,21 @@ struct RopeParams {
 struct LaunchRecord {
     int kernel = QKR_KERNEL_NONE;
     int lanes_per_row = 0, slots = 0, tokens_per_cta = 0, heads_per_item = 0, cluster = 1,
-        block = 0;
+        block = 0, pipelined = 0;
     int64_t grid = 0, launches = 0;
 };
 
-// Launch-shape override of the rope kernels (0: automatic).
-void set_rope_shape_override(int heads_per_item, int tokens_per_cta);
+// Launch-shape override of the rope kernels (0: automatic); pipeline: 0 auto,
+// 1 register kernel only, 2 bulk-copy pipelined kernel only.
+void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta);
+
+// Bulk-copy pipelined rope kernel (rope_tma.cu); cudaErrorNotSupported when a
+// call is outside what it serves.
+cudaError_t launch_rope_tma(const RopeParams &p, int layout_paired, int lpr, int ns,
+                            int tokens_per_tile, cudaStream_t stream, LaunchRecord *rec);
+// Reads (and optionally clears) the device status word that bounded waits set
+// on timeout.  Synchronous.
+cudaError_t read_device_status(unsigned *status, bool reset);
 
 // Each launcher enqueues exactly one kernel and returns the CUDA launch status.
 cudaError_t launch_rope_rows(const RopeParams &p, int pairing, cudaStream_t stream,

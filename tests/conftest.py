@@ -20,3 +20,18 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _device_status_clean(request):
+    """After every GPU test the library's device status word must be 0 (no
+    bounded wait ran out)."""
+    yield
+    if "gpu" not in request.keywords:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import mrope_qk_norm_b200 as qkr
+    torch.cuda.synchronize()
+    assert qkr.device_status(reset=True) == 0, "a kernel wait ran out of its time budget"

@@ -208,3 +208,77 @@ def test_empty_streams():
     g = torch.ones(64, dtype=torch.bfloat16, device="cuda")
     qkr.fused_qk_norm_rope([(e, e, g, g)], e, e, 64, 0, 1e-6, a)
     assert qkr.last_launch()["launches"] == 0
+
+
+def _both_kernels(w, flags=0):
+    """Run once with the bulk-copy pipelined kernel and once with the register
+    kernel; return both results and the two launch records."""
+    try:
+        qkr.tune_rope(2, 0, 0)
+        a = run_fused(w, flags)
+        ia = qkr.last_launch()
+        qkr.tune_rope(1, 0, 0)
+        b = run_fused(w, flags)
+        ib = qkr.last_launch()
+    finally:
+        qkr.tune_rope(0, 0, 0)
+    return a, b, ia, ib
+
+
+@pytest.mark.parametrize("case", ["joint-gptj", "joint-neox", "vit-d80", "partial-tile", "d256"])
+def test_pipelined_equals_register_kernel(case):
+    if case == "joint-gptj":
+        w = W.config3(seed=61, T_txt=77, img_h=9, img_w=13, H=24, D=128, pairing=W.PAIRING_GPTJ)
+    elif case == "joint-neox":
+        w = W.config3(seed=62, T_txt=64, img_h=8, img_w=8, H=24, D=128, pairing=W.PAIRING_NEOX)
+    elif case == "vit-d80":
+        pos = np.random.default_rng(3).integers(0, 4096, (1, 301)).astype(np.int32)
+        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=W.inv_freq(1e4, 32, 64).numpy())
+        w = W.random_rope_case(63, [301], 16, 16, 80, 64, W.PAIRING_NEOX, A)
+    elif case == "partial-tile":
+        pos = np.arange(7, dtype=np.int32)[None]
+        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=W.inv_freq(1e4, 32, 64).numpy())
+        w = W.random_rope_case(64, [7], 3, 1, 64, 64, W.PAIRING_GPTJ, A)
+    else:
+        pos = np.random.default_rng(4).integers(0, 9000, (1, 53)).astype(np.int32)
+        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=W.inv_freq(1e4, 128, 256).numpy())
+        w = W.random_rope_case(65, [53], 4, 2, 256, 256, W.PAIRING_NEOX, A)
+    (qa, ka), (qb, kb), ia, ib = _both_kernels(w)
+    assert ia["pipelined"] == 1 and ib["pipelined"] == 0
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(qa, rq, case + " q")
+    assert_bf16_close(ka, rk, case + " k")
+
+
+def test_pipelined_strided_heads_and_tile_sweep():
+    # non-dense head stride (one bulk copy per row) and every tile size
+    g = torch.Generator().manual_seed(66)
+    T, H, D = 41, 6, 128
+    qkv = W.bf16_normal((T, H, 3, D), g)
+    gq = W.bf16_uniform((D,), 0.5, 1.5, g)
+    gk = W.bf16_uniform((D,), 0.5, 1.5, g)
+    inv = W.inv_freq(1e4, 64, 128)
+    pos = torch.arange(T, dtype=torch.int32).view(1, T) * 3
+    dq = to_dev(qkv)
+    qv = dq[:, :, 0]  # [T, H, D] with head stride 3*D
+    kv = dq[:, :, 1]
+    assert qv.stride(1) == 3 * D
+    a = qkr.angle_positions(to_dev(pos), to_dev(inv))
+    outs = []
+    try:
+        for pipe, tt in [(1, 0), (2, 1), (2, 2), (2, 3), (2, 4)]:
+            qkr.tune_rope(pipe, 0, tt)
+            qo = torch.empty(T, H, D, dtype=torch.bfloat16, device="cuda")
+            ko = torch.empty_like(qo)
+            qkr.fused_qk_norm_rope([(qv, kv, to_dev(gq), to_dev(gk))], qo, ko, D, W.PAIRING_NEOX,
+                                   1e-6, a)
+            torch.cuda.synchronize()
+            assert qkr.last_launch()["pipelined"] == (1 if pipe == 2 else 0)
+            outs.append((qo, ko))
+    finally:
+        qkr.tune_rope(0, 0, 0)
+    for qo, ko in outs[1:]:
+        assert torch.equal(qo.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(ko.view(torch.int16), outs[0][1].view(torch.int16))
