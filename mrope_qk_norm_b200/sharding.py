@@ -1,0 +1,19 @@
+"""Token-range sharding of the normalise-then-rotate path across ranks.
+
+Tokens are independent, so a batch splits into contiguous token ranges, one
+per rank, with no exchange step.  A shard is exactly a chunked launch
+(llama.cpp fork #286, "The change": a launch over a token chunk keeps the
+whole positions buffer and is told where its tokens start): rank r processes
+tokens [t0, t1) of its inputs and passes ``token_offset = t0`` so angles are
+read for the right tokens.
+"""
+from __future__ import annotations
+
+
+def shard_range(n_tokens: int, rank: int, world: int) -> tuple[int, int]:
+    """[t0, t1) of rank `rank` out of `world`: contiguous, sizes differ by <= 1."""
+    if world < 1 or not 0 <= rank < world or n_tokens < 0:
+        raise ValueError("need 0 <= rank < world and n_tokens >= 0")
+    base, extra = divmod(n_tokens, world)
+    t0 = rank * base + min(rank, extra)
+    return t0, t0 + base + (1 if rank < extra else 0)
