@@ -163,21 +163,80 @@ class FusedSet:
 
 
 def time_launches(fns, steps, warmup, stream):
-    """Run fns[i % len] `steps` times; returns (total_ms, per-launch ms list)."""
-    for i in range(warmup):
-        fns[i % len(fns)]()
+    """Run fns[i % len] `steps` times; returns (total_ms, per-launch ms list).
+
+    The `steps` launches are captured into one CUDA graph and replayed once,
+    so host-side call overhead (a few us per ctypes call) does not hide the
+    device time of small kernels; per-launch time is the graph time / steps.
+    """
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, len(fns))):
+            fns[i % len(fns)]()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            fns[i % len(fns)]()
+    with torch.cuda.stream(stream):
+        g.replay()  # untimed replay: first replay uploads the graph
+    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(steps):
-        ev[i][0].record(stream)
-        fns[i % len(fns)]()
-        ev[i][1].record(stream)
-    end.record(stream)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        g.replay()
+        end.record(stream)
     torch.cuda.synchronize()
-    return start.elapsed_time(end), [a.elapsed_time(b) for a, b in ev]
+    total = start.elapsed_time(end)
+    del g
+    return total, [total / steps] * steps
+
+
+def _cudart():
+    """The CUDA runtime torch already loaded (for a plain cudaMemcpyAsync)."""
+    import ctypes
+    import glob
+    for cand in ["libcudart.so.12"] + glob.glob(os.path.join(
+            os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib", "libcudart.so*")):
+        try:
+            return ctypes.CDLL(cand)
+        except OSError:
+            continue
+    raise OSError("libcudart not found")
+
+
+def same_size_copy_us(nbytes: int, dev, stream, steps: int = 200) -> float:
+    """Device time of a device-to-device cudaMemcpyAsync moving the same total
+    bytes (nbytes/2 read + nbytes/2 written), over rotating buffers larger than
+    L2: the practical ceiling for a launch of this size (ramp and tail
+    included).  Timed eagerly: a memcpy node inside a CUDA graph runs on a copy
+    engine at about half this rate, while an eager same-device copy runs as a
+    kernel on the SMs."""
+    import ctypes
+    rt = _cudart()
+    rt.cudaMemcpyAsync.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                   ctypes.c_int, ctypes.c_void_p]
+    half = (nbytes // 2) // 16 * 16
+    nset = n_sets_for(nbytes)
+    src = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nset)]
+    dst = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nset)]
+    sh = stream.cuda_stream
+
+    def cp(i):
+        if rt.cudaMemcpyAsync(dst[i].data_ptr(), src[i].data_ptr(), half, 3, sh) != 0:
+            raise RuntimeError("cudaMemcpyAsync failed")
+    for i in range(10):
+        cp(i % nset)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            cp(i % nset)
+        end.record(stream)
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    del src, dst
+    return 1e3 * total / steps
 
 
 def n_sets_for(bytes_per_set: int) -> int:
@@ -186,12 +245,18 @@ def n_sets_for(bytes_per_set: int) -> int:
 
 # ------------------------------------------------------------- other rows --
 
-def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20):
-    """Each remaining kernel of the path at its own workload."""
+def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
+    """Each remaining kernel of the path at its own workload (`only`: keep the
+    rows whose workload text contains this substring)."""
     import mrope_qk_norm_b200 as qkr
     rows = []
 
+    def want(workload):
+        return only is None or only in workload
+
     def record(name, workload, fns, nbytes, units, unit_name, extra=None):
+        if not want(workload):
+            return
         total, per = time_launches(fns, steps, warmup, stream)
         us = 1e3 * statistics.mean(per)
         gbs = nbytes / (us * 1e-6) / 1e9
@@ -274,7 +339,10 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20):
            apply_bytes, N, "tokens")
 
     # config 2: RMSNorm + residual, decode rows and sweep points
-    for R, hidden in [(1, 5120), (32, 5120), (1024, 8192), (16384, 8192), (16384, 2048)]:
+    for R, hidden in [(1, 5120), (32, 5120), (1024, 8192), (4096, 8192), (16384, 8192),
+                      (16384, 2048)]:
+        if not want("R=%d hidden=%d" % (R, hidden)):
+            continue
         nb = 8 * R * hidden + 2 * hidden
         nset = n_sets_for(nb)
         sets = []
@@ -358,7 +426,7 @@ def reference_arm(args) -> dict:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-kernel rows")
@@ -366,6 +434,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--row-steps", type=int, default=200)
     ap.add_argument("--row-warmup", type=int, default=20)
+    ap.add_argument("--rows-filter", default=None,
+                    help="measure only the rows whose workload contains this text")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -390,7 +460,7 @@ def main():
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                     device_id=dev)
         dist = dist_mod
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)  # graphs are captured on a non-default stream
 
     w = W.config3()  # GPT-J pairing, full size
     nbytes = fused_bytes(512, 4096, 24, 128, 64)
@@ -400,19 +470,36 @@ def main():
 
     sampler = ClockSampler(dev)
     sampler.start()
-    for i in range(args.warmup):
-        fns[i % n_sets]()
+    # warm-up (untimed), then K steps captured in one graph and replayed once
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            fns[i % n_sets]()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            fns[i % n_sets]()
+    with torch.cuda.stream(stream):
+        graph.replay()  # untimed: uploads the graph
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
-    total_ms, per = time_launches(fns, args.steps, 0, stream)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        graph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
     t_wall1 = time.perf_counter()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.stop()
+    total_ms = ev0.elapsed_time(ev1)
+    per = [total_ms / args.steps]
+    del graph
     info = qkr.last_launch()
 
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -424,6 +511,8 @@ def main():
     value = world * tokens / (ms_per_step * 1e-3)
     kern_ms = statistics.mean(per)
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
+
+    copy_us = same_size_copy_us(nbytes, dev, stream)
 
     # end to end: pinned host inputs -> device -> kernel -> pinned host outputs
     host_in = []
@@ -448,16 +537,18 @@ def main():
         host_out[0].copy_(e2e_set.qo, non_blocking=True)
         host_out[1].copy_(e2e_set.ko, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
+    with torch.cuda.stream(stream):  # copies and kernel on one stream, in order
+        for _ in range(3):
+            e2e_step()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
     torch.cuda.synchronize()
     te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
     if dist:
@@ -469,7 +560,8 @@ def main():
     if not args.no_rows:
         del sets, fns
         torch.cuda.empty_cache()
-        rows = measure_rows(dev, stream, peaks["hbm_gbs"], args.row_steps, args.row_warmup)
+        rows = measure_rows(dev, stream, peaks["hbm_gbs"], args.row_steps, args.row_warmup,
+                            args.rows_filter)
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -505,6 +597,8 @@ def main():
                      "algorithmic_bytes_per_launch": nbytes,
                      "kernel_us_per_launch": round(kern_ms * 1e3, 3),
                      "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
+                     "same_size_d2d_copy_us": round(copy_us, 3),
+                     "frac_of_same_size_copy": round(copy_us / (kern_ms * 1e3), 4),
                      "kernel": info.get("kernel_name")},
         "cpu_baseline": cb,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

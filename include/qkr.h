@@ -283,7 +283,8 @@ typedef struct qkr_launch_info {
     int32_t lanes_per_row;   /* rope kernels: lanes that share one head row */
     int32_t slots;           /* rope: 16-byte vectors per lane per row; rms: per thread */
     int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
-    int32_t heads_per_item;  /* rope: head rows a lane group loads together */
+    int32_t heads_per_item;  /* rope: head rows of one token a lane group loads
+                                together (pipelined kernel: head slots per CTA) */
     int32_t pipelined;       /* rope: 1 if rows were staged by bulk copies into a
                                 shared-memory ring (warp-specialised kernel) */
     int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
@@ -296,7 +297,7 @@ qkr_status qkr_last_launch(qkr_launch_info *info);
 /* Launch-shape override for the rope kernels, for tuning sweeps.  pipeline:
  * 0 automatic, 1 register kernel only, 2 bulk-copy pipelined kernel only
  * (calls it cannot serve then fail with QKR_ERR_CUDA); heads per work item
- * (1..8, register kernel) and tokens per CTA or per pipeline tile (1..32);
+ * (1..4, register kernel) and tokens per CTA or per pipeline tile (1..16);
  * 0 keeps the automatic choice.  Process-wide.  Every shape computes
  * bit-identical results: a row's arithmetic does not depend on it.
  * Returns QKR_ERR_INVALID_ARG out of range. */

@@ -343,10 +343,10 @@ qkr_status qkr_last_launch(qkr_launch_info *info)
 
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta)
 {
-    if (pipeline < 0 || pipeline > 2 || heads_per_item < 0 || heads_per_item > 8 ||
-        tokens_per_cta < 0 || tokens_per_cta > 32)
+    if (pipeline < 0 || pipeline > 2 || heads_per_item < 0 || heads_per_item > 4 ||
+        tokens_per_cta < 0 || tokens_per_cta > 16)
         return fail(QKR_ERR_INVALID_ARG,
-                    "pipeline in [0, 2], heads_per_item in [0, 8], tokens_per_cta in [0, 32]");
+                    "pipeline in [0, 2], heads_per_item in [0, 4], tokens_per_cta in [0, 16]");
     qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta);
     g_error.clear();
     return QKR_OK;

@@ -103,7 +103,6 @@ struct RopeParams {
     int Hq, Hk, D, rot, P;
     int rows_per_token;       // Hq + Hk
     int tokens_per_cta;
-    int heads_per_item;       // heads of one token and kind a lane group processes together
     int pw;                   // (cos, sin) columns staged per token: P, or D/2 for GPT-J
                               // (pairs in [P, D/2) get the identity (1, 0))
     float eps, inv_D;
