@@ -52,7 +52,8 @@ def measured_peaks() -> dict:
 
 
 def kernel_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    """DRAM bytes per launch from the committed ncu summary, if still current
+    (the sha256 over the kernel's sources must match the captured build)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -61,9 +62,11 @@ def kernel_traffic(kernel: str):
     e = d.get(kernel)
     if not e:
         return None
-    src = os.path.join(ROOT, e["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    return e["dram_bytes_per_launch"] if h == e["source_sha256"] else None
+    h = hashlib.sha256()
+    for src in e["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    return e["dram_bytes_per_launch"] if h.hexdigest() == e["sources_sha256"] else None
 
 
 # ----------------------------------------------------------------- clocks --
