@@ -361,6 +361,46 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
     return rows
 
 
+def rms_sweep(dev, stream, peak_gbs, steps=100, warmup=5, bar=0.70) -> dict:
+    """RMSNorm + residual over R = 1, 2, 4, ..., 16384 rows x hidden {2048,
+    4096, 8192}.  Inputs are N(0,1) bf16 drawn on the device from a seeded
+    generator (timing only; parity runs on the CPU-generated configs), with
+    enough rotating sets that every launch reads from HBM.  Reports per point
+    (R, us per launch, GB/s, fraction of measured HBM) and, per hidden size,
+    the smallest R reaching `bar` of the measured copy bandwidth."""
+    import mrope_qk_norm_b200 as qkr
+    g = torch.Generator(device=dev)
+    out = {"points": {}, "crossover_R": {}, "bar": bar}
+    for hidden in (2048, 4096, 8192):
+        pts = []
+        cross = None
+        for e in range(15):
+            R = 1 << e
+            nb = 8 * R * hidden + 2 * hidden
+            sets = []
+            for i in range(n_sets_for(nb)):
+                g.manual_seed(1000 * hidden + 100 * e + i)
+                x = torch.randn(R, hidden, device=dev, generator=g).to(torch.bfloat16)
+                r = torch.randn(R, hidden, device=dev, generator=g).to(torch.bfloat16)
+                gm = (0.5 + torch.rand(hidden, device=dev, generator=g)).to(torch.bfloat16)
+                sets.append((x, r, gm, torch.empty_like(x)))
+            total, _ = time_launches(
+                [lambda s=s: qkr.rms_norm_residual(s[0], s[1], s[2], s[3], 1e-6, stream)
+                 for s in sets], steps, warmup, stream)
+            us = 1e3 * total / steps
+            gbs = nb / (us * 1e-6) / 1e9
+            frac = gbs / peak_gbs
+            pts.append([R, round(us, 3), round(gbs, 1), round(frac, 4)])
+            if cross is None and frac >= bar:
+                cross = R
+            del sets
+        out["points"][str(hidden)] = pts
+        out["crossover_R"][str(hidden)] = cross
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------- CPU oracle --
 
 N_IMG_SAMPLE = 512
@@ -437,6 +477,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--row-steps", type=int, default=200)
     ap.add_argument("--row-warmup", type=int, default=20)
+    ap.add_argument("--no-rms-sweep", action="store_true",
+                    help="skip the RMSNorm R x hidden sweep")
     ap.add_argument("--rows-filter", default=None,
                     help="measure only the rows whose workload contains this text")
     args = ap.parse_args()
@@ -565,6 +607,9 @@ def main():
         torch.cuda.empty_cache()
         rows = measure_rows(dev, stream, peaks["hbm_gbs"], args.row_steps, args.row_warmup,
                             args.rows_filter)
+    sweep = None
+    if not args.no_rows and not args.no_rms_sweep and world == 1:
+        sweep = rms_sweep(dev, stream, peaks["hbm_gbs"])
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -610,6 +655,7 @@ def main():
         "gpu_launches": args.steps,
         "clocks": clocks,
         "rows": rows,
+        "rms_sweep": sweep,
     }
     print(json.dumps(line))
     return 0

@@ -289,15 +289,31 @@ typedef struct qkr_launch_info {
                                 shared-memory ring (warp-specialised kernel) */
     int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
     int32_t block;           /* threads per CTA */
+    int32_t direct_angles;   /* rope: 1 if each work item read its (cos, sin) straight
+                                from the fp32 table (16-byte loads), 0 if the angles
+                                were staged per token in shared memory */
+    int32_t overlap;         /* 1 if launched with programmatic stream serialisation
+                                (see qkr_launch_overlap) */
     int64_t grid;            /* CTAs launched */
     int64_t launches;        /* kernel launches enqueued (0 for an empty call) */
 } qkr_launch_info;
 qkr_status qkr_last_launch(qkr_launch_info *info);
 
+/* Programmatic dependent launch for every kernel of this library (default 1).
+ * With 1, a kernel is launched with programmatic stream serialisation: it
+ * may become resident while the previous kernel of the stream drains, and
+ * its first action is a grid-dependency wait that returns once the previous
+ * kernel has completed and its writes are visible; stream order therefore
+ * holds exactly as without it, and results are bit-identical.  What it saves
+ * is the launch gap between back-to-back kernels.  0 launches plainly.
+ * Process-wide.  Returns QKR_ERR_INVALID_ARG for other values. */
+qkr_status qkr_launch_overlap(int32_t enable);
+
 /* Launch-shape override for the rope kernels, for tuning sweeps.  pipeline:
  * 0 automatic, 1 register kernel only, 2 bulk-copy pipelined kernel only
  * (calls it cannot serve then fail with QKR_ERR_CUDA); heads per work item
- * (1..4, register kernel) and tokens per CTA or per pipeline tile (1..16);
+ * (1..4, register kernel) and tokens per CTA or per pipeline tile (1..64;
+ * the staged-angle kernels cap it by their shared memory);
  * 0 keeps the automatic choice.  Process-wide.  Every shape computes
  * bit-identical results: a row's arithmetic does not depend on it.
  * Returns QKR_ERR_INVALID_ARG out of range. */

@@ -29,7 +29,7 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
 
 EXPORTS = ("fused_qk_norm_rope", "mrope_apply", "vit_mrope_setup", "rms_norm_residual",
            "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
-           "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status")
+           "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status", "qkr_launch_overlap")
 
 
 class QkrError(RuntimeError):
@@ -62,6 +62,7 @@ class LaunchInfo(ctypes.Structure):
                 ("slots", ctypes.c_int32), ("tokens_per_cta", ctypes.c_int32),
                 ("heads_per_item", ctypes.c_int32), ("pipelined", ctypes.c_int32),
                 ("cluster", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("direct_angles", ctypes.c_int32), ("overlap", ctypes.c_int32),
                 ("grid", ctypes.c_int64), ("launches", ctypes.c_int64)]
 
 
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "qkr_section_map": [V, I32, V, I64, V],
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
         "qkr_tune_rope": [I32, I32, I32],
+        "qkr_launch_overlap": [I32],
         "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
     }
     for name, args in sig.items():
@@ -152,6 +154,11 @@ def _ptr_base(t, dtype, what):
 def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 0) -> None:
     """Override the rope kernels' launch shape (0 = automatic), for tuning."""
     _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta))
+
+
+def launch_overlap(enable: bool) -> None:
+    """Programmatic dependent launch for every kernel of the library (default on)."""
+    _check(_lib.qkr_launch_overlap(1 if enable else 0))
 
 
 def device_status(reset: bool = False) -> int:

@@ -4,12 +4,21 @@
 // refuses (never degrades) when it cannot serve a call exactly; it never
 // allocates, frees or synchronises.
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
 #include <string>
 
 #include "qkr_internal.cuh"
+
+namespace qkr {
+namespace {
+std::atomic<int> g_overlap{1};
+}
+int launch_overlap() { return g_overlap.load(std::memory_order_relaxed); }
+void set_launch_overlap(int enable) { g_overlap.store(enable ? 1 : 0); }
+}  // namespace qkr
 
 namespace {
 
@@ -150,6 +159,10 @@ qkr_status check_angle(const qkr_angle_desc *a, int64_t P, int64_t T, qkr::RopeP
         p.sin = a->sin;
         p.ld = a->ld;
         p.plane_stride = a->plane_stride;
+        // four consecutive pairs of a row in one 16-byte load when every row
+        // (and plane) start keeps 16-byte alignment
+        p.tab_vec4 = aligned16(a->cos) && aligned16(a->sin) && a->ld % 4 == 0 &&
+                     (planes == 1 || a->plane_stride % 4 == 0);
     } else {
         return fail(QKR_ERR_INVALID_ARG, "unknown angle kind %d", a->kind);
     }
@@ -336,17 +349,28 @@ qkr_status qkr_last_launch(qkr_launch_info *info)
     info->pipelined = g_last.pipelined;
     info->cluster = g_last.cluster;
     info->block = g_last.block;
+    info->direct_angles = g_last.direct_angles;
+    info->overlap = g_last.launches > 0 ? qkr::launch_overlap() : 0;
     info->grid = g_last.grid;
     info->launches = g_last.launches;
+    return QKR_OK;
+}
+
+qkr_status qkr_launch_overlap(int32_t enable)
+{
+    if (enable != 0 && enable != 1)
+        return fail(QKR_ERR_INVALID_ARG, "enable must be 0 or 1");
+    qkr::set_launch_overlap(enable);
+    g_error.clear();
     return QKR_OK;
 }
 
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta)
 {
     if (pipeline < 0 || pipeline > 2 || heads_per_item < 0 || heads_per_item > 4 ||
-        tokens_per_cta < 0 || tokens_per_cta > 16)
+        tokens_per_cta < 0 || tokens_per_cta > 64)
         return fail(QKR_ERR_INVALID_ARG,
-                    "pipeline in [0, 2], heads_per_item in [0, 4], tokens_per_cta in [0, 16]");
+                    "pipeline in [0, 2], heads_per_item in [0, 4], tokens_per_cta in [0, 64]");
     qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta);
     g_error.clear();
     return QKR_OK;

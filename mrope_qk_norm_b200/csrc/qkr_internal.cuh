@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/qkr.h"
 
 namespace qkr {
@@ -54,6 +56,60 @@ __device__ __forceinline__ void st_stream(void *p, const uint4 &v)
 __device__ __forceinline__ uint4 ld_reuse(const void *p)
 {
     return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// ------------------------------------------------ programmatic dependency --
+// A kernel launched with programmatic stream serialisation may begin while
+// the previous kernel of the stream is still draining (its CTAs get resident
+// and wait), instead of after it has fully retired.  Every library kernel
+// calls pdl_wait() before its first global-memory access: the wait returns
+// once the previous grid has completed and its writes are visible, so the
+// usual stream ordering holds for everything the kernel reads or writes.
+// pdl_trigger() lets the next dependent launch begin scheduling.  Both are
+// no-ops for a kernel launched without the attribute.  The wait is the
+// hardware's grid-completion dependency (like a stream dependency), not a
+// software spin on a flag.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Process-wide switch (qkr_launch_overlap); 1 = launch with the attribute.
+int launch_overlap();
+void set_launch_overlap(int enable);
+
+// Launch `fn` on `stream` with the programmatic-serialisation attribute when
+// the switch is on, plus an optional cluster dimension (cluster_x > 1).
+template <typename... Params, typename... Args>
+cudaError_t launch(void (*fn)(Params...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t stream, int cluster_x, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (launch_overlap()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------ section rule --
@@ -115,13 +171,14 @@ struct RopeParams {
     const float *cos;
     const float *sin;
     int64_t ld, plane_stride;
+    int tab_vec4;             // table bases 16-byte aligned, ld and plane_stride % 4 == 0
     int64_t token_offset;
 };
 
 struct LaunchRecord {
     int kernel = QKR_KERNEL_NONE;
     int lanes_per_row = 0, slots = 0, tokens_per_cta = 0, heads_per_item = 0, cluster = 1,
-        block = 0, pipelined = 0;
+        block = 0, pipelined = 0, direct_angles = 0;
     int64_t grid = 0, launches = 0;
 };
 

@@ -111,6 +111,8 @@ __device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int
 template <int VPT>
 __global__ void __launch_bounds__(kMaxThreads) rms_rows_kernel(const __grid_constant__ RmsParams p)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[32];
     const int64_t row = blockIdx.x;
     float s[VPT][8];
@@ -126,6 +128,8 @@ template <int VPT>
 __global__ void __launch_bounds__(kMaxThreads)
 rms_cluster_kernel(const __grid_constant__ RmsParams p)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float red[32];
     __shared__ float partial;
     cg::cluster_group cluster = cg::this_cluster();
@@ -221,8 +225,7 @@ cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, La
 
     cudaError_t err;
     if (cs == 1) {
-        rows_fn(vpt)<<<(unsigned)grid, threads, 0, stream>>>(p);
-        err = cudaGetLastError();
+        err = launch(rows_fn(vpt), dim3((unsigned)grid), dim3(threads), 0, stream, 1, p);
     } else {
         Fn fn = cluster_fn(vpt);
         if (cs > 8) {
@@ -230,19 +233,7 @@ cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, La
             if (err != cudaSuccess)
                 return err;
         }
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)grid);
-        cfg.blockDim = dim3(threads);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = cs;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, fn, p);
+        err = launch(fn, dim3((unsigned)grid), dim3(threads), 0, stream, cs, p);
     }
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();

@@ -1,0 +1,442 @@
+// rope_fast.cuh -- the item-based per-head RMSNorm + RoPE / mRoPE kernel.
+//
+// One kernel template serves fused_qk_norm_rope (vllm-omni #7600: per-stream
+// per-head RMSNorm of Q and K, text-first concatenation and RoPE in one
+// launch) and mrope_apply (llama.cpp fork #286: each rotated pair reads the
+// position row its section selects; a chunk reads the whole positions buffer
+// from a token offset).  Its instantiations are split over several
+// translation units (rope_fast_*.cu) so they compile in parallel; each unit
+// exports one picker.
+//
+// B200 mapping.  The op moves ~4 bytes per element and does a handful of
+// flops on it, so it is HBM-bound only if the instruction stream stays lean:
+//   * a CTA owns a balanced range of consecutive joint tokens and all of
+//     their Q and K heads; the grid is sized to the device (one wave of
+//     resident CTAs for the direct-angle kernels), so every SM gets the same
+//     share of rows and the last wave is not left half empty;
+//   * a work item is (token, Q or K, a block of U heads).  A group of LPR
+//     lanes takes an item, loads the (cos, sin) of its pairs and the gamma of
+//     its columns into registers once, and issues the 16-byte loads of all U
+//     rows before any math (U * slots * 16 bytes in flight per lane);
+//   * staged angles: each token's (cos, sin) is computed once (sincosf of
+//     the fp32 position x inv_freq product) or read once from the table into
+//     shared memory, and every head of the token reuses it.  Direct angles
+//     (an fp32 table whose rows allow 16-byte reads of four pairs): every
+//     item reads its token's row straight from the table (L1/L2 serve the
+//     other heads), so the kernel has no staging prologue and no block
+//     barrier, and a CTA's table and row loads are in flight together;
+//   * the math runs on Blackwell's packed fp32x2 instructions (FFMA2 / FMUL2)
+//     with each float2 holding the first members of two pairs (A) or the
+//     second members (B): rotation is A' = A C - B S, B' = B C + A S for
+//     NeoX and GPT-J alike, so no lane ever needs another lane's data;
+//   * NeoX with rot_dim % 16 == 0 (PAIRED layout): a lane loads vector u of
+//     the first rotary half and vector u + rot/16 of the second half;
+//     GPT-J (VECTOR layout): pairs (2j, 2j+1) sit in one 32-bit word, and two
+//     words make one (A, B) float2 couple; pairs past rot_dim take (1, 0), so
+//     they pass through exactly with no branch;
+//   * the fp32 sum of squares is reduced with xor shuffles inside the group;
+//     every loop trip count is uniform across a warp so the full-mask
+//     shuffles are always complete.
+// Addresses are 64-bit throughout (large storage offsets, vllm-omni #7600).
+#pragma once
+
+#include "qkr_internal.cuh"
+
+namespace qkr {
+
+using KernelFn = void (*)(RopeParams);
+
+// Pickers exported by the instantiation units: layout and angle path (staged
+// or direct) fixed by the unit; lanes per row, slots, heads per item and the
+// norm flags chosen at run time.
+KernelFn pick_fast_paired_staged(int lpr, int ns, int u, bool norm, bool round);
+KernelFn pick_fast_paired_direct(int lpr, int ns, int u, bool norm, bool round);
+KernelFn pick_fast_vector_staged(int lpr, int ns, int u, bool norm, bool round);
+KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, bool round);
+
+namespace {
+
+constexpr int kThreads = 256;
+
+enum Layout { PAIRED = 0, VECTOR = 1, EXCHANGE = 2 };
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
+
+__device__ __forceinline__ uint32_t word(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ void set_word(uint4 &v, int i, uint32_t w)
+{
+    if (i == 0) v.x = w;
+    else if (i == 1) v.y = w;
+    else if (i == 2) v.z = w;
+    else v.w = w;
+}
+
+__device__ __forceinline__ float2 round2_bf16(float2 a)
+{
+    const uint32_t w = pack2(a.x, a.y);
+    return f2(bf_lo(w), bf_hi(w));
+}
+
+// Stage (cos, sin) of `ntok` tokens into shared memory, SoA, row stride cs_ld.
+// Columns [P, pw) get the identity rotation (1, 0).
+__device__ __forceinline__ void stage_angles(const RopeParams &p, int64_t tok0, int ntok,
+                                             int cs_ld, float *cosv, float *sinv)
+{
+    const int pw = p.pw;
+    for (int idx = threadIdx.x; idx < ntok * pw; idx += kThreads) {
+        const int tt = idx / pw;
+        const int j = idx - tt * pw;
+        float c = 1.f, s = 0.f;
+        if (j < p.P) {
+            const int64_t n = p.token_offset + tok0 + tt;
+            const int axis = section_axis(p.section_mode, p.sec, j);
+            if (p.angle_kind == QKR_ANGLE_POSITIONS) {
+                const int32_t pos = __ldg(p.pos + (int64_t)axis * p.pos_rs + n);
+                const float theta = __fmul_rn((float)pos, __ldg(p.inv_freq + j));
+                sincosf(theta, &s, &c);
+            } else {
+                const int64_t at = (int64_t)axis * p.plane_stride + n * p.ld + j;
+                c = __ldg(p.cos + at);
+                s = __ldg(p.sin + at);
+            }
+        }
+        cosv[tt * cs_ld + j] = c;
+        sinv[tt * cs_ld + j] = s;
+    }
+}
+
+// (cos, sin) of the four pairs j0 .. j0+3 (j0 % 4 == 0) of token n straight
+// from the fp32 table, one 16-byte load each.  The launcher takes this path
+// only when it is exact: 16-byte aligned rows (tab_vec4), P % 4 == 0 and
+// section boundaries on multiples of 4 under a contiguous (or no) section
+// map, so four pairs never straddle P or a plane change.  Pairs past P take
+// the identity (1, 0).
+__device__ __forceinline__ void table_quad(const RopeParams &p, int64_t n, int j0, float4 &c4,
+                                           float4 &s4)
+{
+    if (j0 < p.P) {
+        const int axis = section_axis(p.section_mode, p.sec, j0);
+        const int64_t at = (int64_t)axis * p.plane_stride + (p.token_offset + n) * p.ld + j0;
+        c4 = __ldg(reinterpret_cast<const float4 *>(p.cos + at));
+        s4 = __ldg(reinterpret_cast<const float4 *>(p.sin + at));
+    } else {
+        c4 = make_float4(1.f, 1.f, 1.f, 1.f);
+        s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// One work item: U consecutive heads of one token's Q or K.
+struct Item {
+    const __nv_bfloat16 *src;  // first head's row
+    __nv_bfloat16 *dst;        // first head's output row
+    int64_t hs;                // source head stride
+    int tt;                    // token within the CTA's tile
+    int nh;                    // heads in this item (0: no work)
+    bool isk;
+    bool s1;                   // second stream
+};
+
+template <int U>
+__device__ __forceinline__ Item decode_item(const RopeParams &p, int64_t tok0, int item,
+                                            int items, int gpt, int nbq)
+{
+    Item r;
+    const bool live = item < items;
+    const int it = live ? item : 0;
+    r.tt = it / gpt;
+    const int b = it - r.tt * gpt;
+    r.isk = b >= nbq;
+    const int h0 = (r.isk ? b - nbq : b) * U;
+    r.nh = live ? min(U, (r.isk ? p.Hk : p.Hq) - h0) : 0;
+    const int64_t n = tok0 + r.tt;
+    r.s1 = n >= p.split;
+    const int64_t t = r.s1 ? n - p.split : n;
+    const RopeStreamDev &S0 = p.st[0];
+    const RopeStreamDev &S1 = p.st[1];
+    const __nv_bfloat16 *base = r.isk ? (r.s1 ? S1.k : S0.k) : (r.s1 ? S1.q : S0.q);
+    const int64_t ts = r.isk ? (r.s1 ? S1.k_ts : S0.k_ts) : (r.s1 ? S1.q_ts : S0.q_ts);
+    r.hs = r.isk ? (r.s1 ? S1.k_hs : S0.k_hs) : (r.s1 ? S1.q_hs : S0.q_hs);
+    r.src = base + t * ts + (int64_t)h0 * r.hs;
+    r.dst = (r.isk ? p.k_out : p.q_out) + n * (r.isk ? p.ko_ts : p.qo_ts) + (int64_t)h0 * p.D;
+    return r;
+}
+
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, bool ROUND, bool DIRECT>
+__global__ void __launch_bounds__(kThreads)
+rope_fast_kernel(const __grid_constant__ RopeParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    // Quads (couples of pairs) per lane: PAIRED lo/hi vectors hold 4, each
+    // VECTOR slot holds 2.  Pass-through slots (PAIRED tail) are scaled only.
+    constexpr int NQ = LAYOUT == PAIRED ? 4 : 2 * NS;
+    constexpr int NT = LAYOUT == PAIRED ? NS - 2 : 0;
+    constexpr int G = kThreads / LPR;
+
+    extern __shared__ float4 smem[];
+    const int cs_ld = (p.pw + 3) & ~3;
+    float *cosv = reinterpret_cast<float *>(smem);
+    float *sinv = cosv + p.tokens_per_cta * cs_ld;
+
+    // CTA c owns joint tokens [c T / grid, (c+1) T / grid): balanced ranges of
+    // at most tokens_per_cta tokens (T < 2^31, checked by the launcher).
+    const int64_t tok0 = (int64_t)blockIdx.x * p.T / gridDim.x;
+    const int ntok = (int)((int64_t)(blockIdx.x + 1) * p.T / gridDim.x - tok0);
+    if (!DIRECT) {
+        stage_angles(p, tok0, ntok, cs_ld, cosv, sinv);
+        __syncthreads();
+    }
+
+    const int lane = threadIdx.x % LPR;
+    const int grp = threadIdx.x / LPR;
+    const int D = p.D;
+    const int nvec = D >> 3;
+    const int npv = p.rot >> 4;
+    // vector index of each slot (-1: none)
+    int vidx[NS];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        int v;
+        if (LAYOUT == PAIRED)
+            v = k == 0 ? (lane < npv ? lane : -1)
+              : k == 1 ? (lane < npv ? lane + npv : -1)
+                       : 2 * npv + lane + LPR * (k - 2);
+        else
+            v = lane + LPR * k;
+        vidx[k] = (v >= 0 && v < nvec) ? v : -1;
+    }
+    // first pair index of each quad
+    int qpair[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+        qpair[q] = LAYOUT == PAIRED ? 8 * lane + 2 * q : 4 * (lane + LPR * (q >> 1)) + 2 * (q & 1);
+
+    const int nbq = (p.Hq + U - 1) / U;
+    const int gpt = nbq + (p.Hk + U - 1) / U;
+    const int items = ntok * gpt;
+
+    for (int it0 = 0; it0 < items; it0 += G) {  // uniform trip count across the CTA
+        const Item m = decode_item<U>(p, tok0, it0 + grp, items, gpt, nbq);
+
+        uint4 raw[U][NS];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                raw[u][k] = (u < m.nh && vidx[k] >= 0)
+                                ? ld_stream(m.src + u * m.hs + 8 * vidx[k])
+                                : make_uint4(0, 0, 0, 0);
+
+        // (cos, sin) of this lane's pairs for the item's token
+        float2 C[NQ], Sn[NQ];
+        {
+            const bool have = LAYOUT == PAIRED ? vidx[0] >= 0 : true;
+#pragma unroll
+            for (int q = 0; q < NQ; q += 2) {
+                const bool ok = m.nh > 0 && have && (LAYOUT == PAIRED || vidx[q >> 1] >= 0);
+                float4 c4 = make_float4(1.f, 1.f, 1.f, 1.f);
+                float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (ok) {
+                    if (DIRECT) {
+                        table_quad(p, tok0 + m.tt, qpair[q], c4, s4);
+                    } else {
+                        c4 = *reinterpret_cast<const float4 *>(cosv + m.tt * cs_ld + qpair[q]);
+                        s4 = *reinterpret_cast<const float4 *>(sinv + m.tt * cs_ld + qpair[q]);
+                    }
+                }
+                C[q] = f2(c4.x, c4.y);
+                C[q + 1] = f2(c4.z, c4.w);
+                Sn[q] = f2(s4.x, s4.y);
+                Sn[q + 1] = f2(s4.z, s4.w);
+            }
+        }
+        // gamma of this lane's columns, in the same (A, B) arrangement
+        float2 GA[NQ], GB[NQ], GT[NT > 0 ? NT : 1][4];
+        if (NORM) {
+            const RopeStreamDev &S = m.s1 ? p.st[1] : p.st[0];
+            const __nv_bfloat16 *gam = m.isk ? S.gk : S.gq;
+            uint4 gv[NS];
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                if (LAYOUT == PAIRED) {
+                    const uint32_t wa = word(gv[0], q), wb = word(gv[1], q);
+                    GA[q] = f2(bf_lo(wa), bf_hi(wa));
+                    GB[q] = f2(bf_lo(wb), bf_hi(wb));
+                } else {
+                    const uint32_t w0 = word(gv[q >> 1], 2 * (q & 1));
+                    const uint32_t w1 = word(gv[q >> 1], 2 * (q & 1) + 1);
+                    GA[q] = f2(bf_lo(w0), bf_lo(w1));
+                    GB[q] = f2(bf_hi(w0), bf_hi(w1));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = word(gv[2 + k], i);
+                    GT[k][i] = f2(bf_lo(w), bf_hi(w));
+                }
+        }
+
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float2 A[NQ], B[NQ], TL[NT > 0 ? NT : 1][4];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                if (LAYOUT == PAIRED) {
+                    const uint32_t wa = word(raw[u][0], q), wb = word(raw[u][1], q);
+                    A[q] = f2(bf_lo(wa), bf_hi(wa));
+                    B[q] = f2(bf_lo(wb), bf_hi(wb));
+                } else {
+                    const uint32_t w0 = word(raw[u][q >> 1], 2 * (q & 1));
+                    const uint32_t w1 = word(raw[u][q >> 1], 2 * (q & 1) + 1);
+                    A[q] = f2(bf_lo(w0), bf_lo(w1));
+                    B[q] = f2(bf_hi(w0), bf_hi(w1));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = word(raw[u][2 + k], i);
+                    TL[k][i] = f2(bf_lo(w), bf_hi(w));
+                }
+
+            if (NORM) {
+                float2 acc = f2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                    acc = __ffma2_rn(A[q], A[q], acc);
+                    acc = __ffma2_rn(B[q], B[q], acc);
+                }
+#pragma unroll
+                for (int k = 0; k < NT; ++k)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        acc = __ffma2_rn(TL[k][i], TL[k][i], acc);
+                float ss = acc.x + acc.y;
+#pragma unroll
+                for (int off = LPR / 2; off > 0; off >>= 1)
+                    ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
+                const float2 r2 = f2(r, r);
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                    A[q] = __fmul2_rn(__fmul2_rn(A[q], r2), GA[q]);
+                    B[q] = __fmul2_rn(__fmul2_rn(B[q], r2), GB[q]);
+                    if (ROUND) {
+                        A[q] = round2_bf16(A[q]);
+                        B[q] = round2_bf16(B[q]);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < NT; ++k)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        TL[k][i] = __fmul2_rn(__fmul2_rn(TL[k][i], r2), GT[k][i]);
+            }
+
+            // rotate: A' = A C - B S, B' = B C + A S (packed over two pairs)
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const float2 bs = __fmul2_rn(B[q], Sn[q]);
+                const float2 bc = __fmul2_rn(B[q], C[q]);
+                const float2 a2 = __ffma2_rn(A[q], C[q], f2(-bs.x, -bs.y));
+                const float2 b2 = __ffma2_rn(A[q], Sn[q], bc);
+                A[q] = a2;
+                B[q] = b2;
+            }
+
+            uint4 outv[NS];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                if (LAYOUT == PAIRED) {
+                    set_word(outv[0], q, pack2(A[q].x, A[q].y));
+                    set_word(outv[1], q, pack2(B[q].x, B[q].y));
+                } else {
+                    set_word(outv[q >> 1], 2 * (q & 1), pack2(A[q].x, B[q].x));
+                    set_word(outv[q >> 1], 2 * (q & 1) + 1, pack2(A[q].y, B[q].y));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    set_word(outv[2 + k], i, pack2(TL[k][i].x, TL[k][i].y));
+
+            if (u < m.nh) {
+#pragma unroll
+                for (int k = 0; k < NS; ++k)
+                    if (vidx[k] >= 0)
+                        st_stream(m.dst + (int64_t)u * D + 8 * vidx[k], outv[k]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------- pickers --
+
+template <int LAYOUT, bool DIRECT, int LPR, int NS, int U>
+KernelFn pick_flags(bool norm, bool round)
+{
+    if (!norm)
+        return rope_fast_kernel<LAYOUT, LPR, NS, U, false, false, DIRECT>;
+    return round ? rope_fast_kernel<LAYOUT, LPR, NS, U, true, true, DIRECT>
+                 : rope_fast_kernel<LAYOUT, LPR, NS, U, true, false, DIRECT>;
+}
+
+template <int LAYOUT, bool DIRECT, int LPR, int NS>
+KernelFn pick_u(int u, bool norm, bool round)
+{
+    switch (u) {
+    case 1: return pick_flags<LAYOUT, DIRECT, LPR, NS, 1>(norm, round);
+    case 2: return pick_flags<LAYOUT, DIRECT, LPR, NS, 2>(norm, round);
+    case 3: return pick_flags<LAYOUT, DIRECT, LPR, NS, 3>(norm, round);
+    case 4: return pick_flags<LAYOUT, DIRECT, LPR, NS, 4>(norm, round);
+    default: return nullptr;
+    }
+}
+
+template <int LAYOUT, bool DIRECT, int LPR>
+KernelFn pick_ns(int ns, int u, bool norm, bool round)
+{
+    if constexpr (LAYOUT == PAIRED) {
+        // slots 0/1: the two rotary halves of the lane's pairs; 2, 3: pass-through tail
+        switch (ns) {
+        case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, round);
+        case 3: return pick_u<LAYOUT, DIRECT, LPR, 3>(u, norm, round);
+        case 4: return pick_u<LAYOUT, DIRECT, LPR, 4>(u, norm, round);
+        default: return nullptr;
+        }
+    } else {
+        switch (ns) {
+        case 1: return pick_u<LAYOUT, DIRECT, LPR, 1>(u, norm, round);
+        case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, round);
+        default: return nullptr;
+        }
+    }
+}
+
+template <int LAYOUT, bool DIRECT>
+KernelFn pick_fast(int lpr, int ns, int u, bool norm, bool round)
+{
+    switch (lpr) {
+    case 1: return pick_ns<LAYOUT, DIRECT, 1>(ns, u, norm, round);
+    case 2: return pick_ns<LAYOUT, DIRECT, 2>(ns, u, norm, round);
+    case 4: return pick_ns<LAYOUT, DIRECT, 4>(ns, u, norm, round);
+    case 8: return pick_ns<LAYOUT, DIRECT, 8>(ns, u, norm, round);
+    case 16: return pick_ns<LAYOUT, DIRECT, 16>(ns, u, norm, round);
+    default: return nullptr;
+    }
+}
+
+}  // namespace
+}  // namespace qkr

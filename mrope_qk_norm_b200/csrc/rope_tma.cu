@@ -169,6 +169,8 @@ template <int LAYOUT, int LPR, int NS, bool NORM, bool ROUND>
 __global__ void __launch_bounds__(kMaxThreads, 2)
 rope_tma_kernel(const __grid_constant__ RopeParams p, const __grid_constant__ TmaGeom tg)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int NQ = LAYOUT == PAIRED ? 4 : 2 * NS;
     constexpr int NT = LAYOUT == PAIRED ? NS - 2 : 0;
 
@@ -632,8 +634,8 @@ cudaError_t launch_rope_tma(const RopeParams &p_in, int layout_paired, int lpr, 
         if (grid_x > n_tiles)
             grid_x = n_tiles;
     }
-    fn<<<dim3((unsigned)grid_x, (unsigned)gy), 32 + n_consumers, smem, stream>>>(p, tg);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch(fn, dim3((unsigned)grid_x, (unsigned)gy), dim3(32 + n_consumers),
+                           smem, stream, 1, p, tg);
     if (e == cudaSuccess && rec) {
         *rec = LaunchRecord();
         rec->kernel = layout == PAIRED ? QKR_KERNEL_ROPE_PAIRED : QKR_KERNEL_ROPE_VECTOR;

@@ -53,6 +53,8 @@ __device__ __forceinline__ void token_position(const int32_t *cu, const int32_t 
 
 __global__ void __launch_bounds__(kThreads) vit_setup_kernel(const __grid_constant__ VitParams p)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int spos[3][kTokens];
     const int64_t n0 = (int64_t)blockIdx.x * kTokens;
     const int ntok = (int)min((int64_t)kTokens, p.N - n0);
@@ -83,6 +85,8 @@ __global__ void __launch_bounds__(kThreads) vit_setup_kernel(const __grid_consta
 
 __global__ void vit_positions_kernel(const __grid_constant__ VitParams p, int32_t *out)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (n >= p.N)
         return;
@@ -101,6 +105,8 @@ struct SectionArgs {
 
 __global__ void section_map_kernel(const __grid_constant__ SectionArgs a, int8_t *out)
 {
+    pdl_wait();
+    pdl_trigger();
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     if (j < a.P)
         out[j] = (int8_t)section_axis(a.mode, a.sec, j);
@@ -113,8 +119,8 @@ cudaError_t launch_vit_setup(const VitParams &p, cudaStream_t stream, LaunchReco
     const int64_t grid = (p.N + kTokens - 1) / kTokens;
     if (grid > INT_MAX)
         return cudaErrorInvalidConfiguration;
-    vit_setup_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(p);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch(vit_setup_kernel, dim3((unsigned)grid), dim3(kThreads), 0, stream,
+                             1, p);
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();
         rec->kernel = QKR_KERNEL_VIT_SETUP;
@@ -132,8 +138,8 @@ cudaError_t launch_vit_positions(const VitParams &p, int32_t *pos_out, cudaStrea
     const int64_t grid = (p.N + kThreads - 1) / kThreads;
     if (grid > INT_MAX)
         return cudaErrorInvalidConfiguration;
-    vit_positions_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(p, pos_out);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch(vit_positions_kernel, dim3((unsigned)grid), dim3(kThreads), 0,
+                             stream, 1, p, pos_out);
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();
         rec->kernel = QKR_KERNEL_VIT_POSITIONS;
@@ -153,8 +159,7 @@ cudaError_t launch_section_map(int mode, const int (&sec)[4], int P, int8_t *out
         a.sec[i] = sec[i];
     a.P = P;
     const int grid = (P + 127) / 128;
-    section_map_kernel<<<grid, 128, 0, stream>>>(a, out);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch(section_map_kernel, dim3(grid), dim3(128), 0, stream, 1, a, out);
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();
         rec->kernel = QKR_KERNEL_SECTION_MAP;

@@ -282,3 +282,107 @@ def test_pipelined_strided_heads_and_tile_sweep():
     for qo, ko in outs[1:]:
         assert torch.equal(qo.view(torch.int16), outs[0][0].view(torch.int16))
         assert torch.equal(ko.view(torch.int16), outs[0][1].view(torch.int16))
+
+
+def _table_call(w, cos, sin, mode=W.SECTIONS_NONE, sections=None):
+    """Run w with the given device tables; returns (q, k, launch record)."""
+    keep = []
+    streams = []
+    for s in w.streams:
+        t = (to_dev(s.q), to_dev(s.k), to_dev(s.gamma_q), to_dev(s.gamma_k))
+        keep += list(t)
+        streams.append(t)
+    T = w.n_tokens
+    qo = Guarded((T, w.Hq, w.D))
+    ko = Guarded((T, w.Hk, w.D))
+    a = qkr.angle_table(cos, sin, mode, sections)
+    qkr.fused_qk_norm_rope(streams, qo.tensor, ko.tensor, w.rot, w.pairing, w.eps, a)
+    torch.cuda.synchronize()
+    qo.check()
+    ko.check()
+    return qo.tensor, ko.tensor, qkr.last_launch()
+
+
+@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
+def test_direct_table_reads_equal_staged(pairing):
+    """Per-item 16-byte table reads and per-token staging give the same bits.
+
+    A table with row pitch 64 floats is read directly; the same values at row
+    pitch 66 (rows no longer 16-byte aligned) are staged in shared memory."""
+    w = W.config3(seed=71, T_txt=45, img_h=7, img_w=9, H=12, D=128, pairing=pairing)
+    cos = to_dev(torch.as_tensor(np.asarray(w.angle.cos), dtype=torch.float32))[0]
+    sin = to_dev(torch.as_tensor(np.asarray(w.angle.sin), dtype=torch.float32))[0]
+    T, P = cos.shape
+    cw = torch.zeros(T, 66, dtype=torch.float32, device="cuda")
+    sw = torch.zeros_like(cw)
+    cw[:, :P] = cos
+    sw[:, :P] = sin
+    qd, kd, ld = _table_call(w, cos, sin)
+    qs, ks, ls = _table_call(w, cw[:, :P], sw[:, :P])
+    assert ld["direct_angles"] == 1 and ls["direct_angles"] == 0
+    assert torch.equal(qd.view(torch.int16), qs.view(torch.int16))
+    assert torch.equal(kd.view(torch.int16), ks.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(qd, rq, "direct q")
+    assert_bf16_close(kd, rk, "direct k")
+
+
+@pytest.mark.parametrize("sections,direct", [((16, 24, 24), 1), ((18, 22, 24), 0),
+                                             ((12, 20, 32), 1), ((30, 2, 32), 0)])
+def test_plane_sections_direct_and_staged(sections, direct):
+    """Three planes under contiguous sections: boundaries on multiples of four
+    pairs are read directly, others are staged; both match the oracle."""
+    rng = np.random.default_rng(sum(sections) * 7 + sections[0])
+    T, H, D, rot = 83, 5, 128, 128
+    P = rot // 2
+    ang = rng.uniform(-40.0, 40.0, (3, T, P))
+    cos = np.cos(ang).astype(np.float32)
+    sin = np.sin(ang).astype(np.float32)
+    A = W.AngleInputs(kind=W.ANGLE_TABLE, cos=cos, sin=sin, section_mode=W.SECTIONS_CONTIGUOUS,
+                      sections=sections)
+    w = W.random_rope_case(81 + sections[0], [T], H, 3, D, rot, W.PAIRING_NEOX, A)
+    q, k, rec = _table_call(w, to_dev(torch.from_numpy(cos)), to_dev(torch.from_numpy(sin)),
+                            W.SECTIONS_CONTIGUOUS, sections)
+    assert rec["direct_angles"] == direct
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(q, rq, "planes q")
+    assert_bf16_close(k, rk, "planes k")
+
+
+def test_direct_table_launch_shapes_bit_identical():
+    """Every (heads per item, token split) shape of the direct-angle kernel
+    computes the same bits, including ranges larger than the staged kernels
+    allow and the automatic one-wave grid."""
+    w = W.config3(seed=73, T_txt=33, img_h=6, img_w=11, H=10, D=128, pairing=W.PAIRING_GPTJ)
+    cos = to_dev(torch.as_tensor(np.asarray(w.angle.cos), dtype=torch.float32))
+    sin = to_dev(torch.as_tensor(np.asarray(w.angle.sin), dtype=torch.float32))
+    outs = []
+    try:
+        for u, tt in [(0, 0), (1, 1), (2, 3), (3, 16), (4, 64)]:
+            qkr.tune_rope(1, u, tt)
+            q, k, rec = _table_call(w, cos, sin)
+            assert rec["direct_angles"] == 1
+            if tt:
+                T = w.n_tokens
+                assert rec["grid"] == -(-T // tt) and rec["heads_per_item"] == u
+                assert rec["tokens_per_cta"] == -(-T // rec["grid"])
+            outs.append((q, k))
+    finally:
+        qkr.tune_rope(0, 0, 0)
+    for q, k in outs[1:]:
+        assert torch.equal(q.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(k.view(torch.int16), outs[0][1].view(torch.int16))
+
+
+def test_one_wave_grid_covers_every_token():
+    """The automatic direct-angle grid is one wave of resident CTAs with
+    balanced token ranges; token counts around multiples of the grid (and
+    fewer tokens than CTAs) still write every row exactly once."""
+    for T_txt, img_w in ((297, 1), (297, 37), (297, 45), (5, 1)):
+        w = W.config3(seed=75 + img_w, T_txt=T_txt, img_h=8, img_w=img_w, H=4, D=64,
+                      pairing=W.PAIRING_GPTJ)
+        q, k, _, _ = check_against_oracle(w, what="one wave T=%d" % w.n_tokens)
+        rec = qkr.last_launch()
+        assert rec["direct_angles"] == 1
+        assert rec["grid"] <= w.n_tokens
+        assert rec["tokens_per_cta"] == -(-w.n_tokens // rec["grid"])
