@@ -243,7 +243,10 @@ def same_size_copy_us(nbytes: int, dev, stream, steps: int = 200) -> float:
 
 
 def n_sets_for(bytes_per_set: int) -> int:
-    return max(1, min(8, -(-2 * L2_BYTES // bytes_per_set) + 1))
+    """Rotating copies so consecutive launches touch more than twice the L2
+    (capped at 64 copies: below ~4 MB per launch a kernel is latency-bound and
+    its buffers stay in L2 whatever the rotation)."""
+    return max(1, min(64, -(-2 * L2_BYTES // bytes_per_set) + 1))
 
 
 # ------------------------------------------------------------- other rows --
@@ -316,7 +319,7 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
            {"launches_per_step": 2})
     del s4
 
-    # config 5: ViT setup and apply
+    # config 5: ViT setup and apply, each over rotating output/input sets
     w5 = W.config5()
     g = np.asarray(w5.grids, dtype=np.int64)
     cu = np.concatenate([[0], np.cumsum(g[:, 0] * g[:, 1] * g[:, 2])])
@@ -325,21 +328,30 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
     G = len(w5.grids)
     cu_d, grids_d = meta[:G + 1], meta[G + 1:].view(G, 3)
     inv_t, inv_h, inv_w = (v.to(dev) for v in (w5.inv_t, w5.inv_h, w5.inv_w))
-    cos5 = torch.empty(3, N, 64, dtype=torch.float32, device=dev)
-    sin5 = torch.empty_like(cos5)
     setup_bytes = 2 * N * 64 * 4 + (G + 1 + 3 * G) * 4 + 64 * 4
+    planes = []
+    for _ in range(n_sets_for(setup_bytes)):
+        cos5 = torch.empty(3, N, 64, dtype=torch.float32, device=dev)
+        planes.append((cos5, torch.empty_like(cos5)))
     record("vit_mrope_setup", "8 grids N=%d, planes (3,N,64) fp32" % N,
-           [lambda: qkr.vit_mrope_setup(inv_t, inv_h, inv_w, cu_d, grids_d, N, 2, cos5, sin5,
-                                        stream)], setup_bytes, N, "tokens")
-    q5, k5 = w5.q.to(dev), w5.k.to(dev)
-    gq5, gk5 = w5.gamma_q.to(dev), w5.gamma_k.to(dev)
-    qo5, ko5 = torch.empty_like(q5), torch.empty_like(k5)
-    a5 = qkr.angle_table(cos5, sin5, W.SECTIONS_CONTIGUOUS, (16, 24, 24))
-    d5 = [qkr.stream_desc(q5, k5, gq5, gk5)]
+           [lambda c=c: qkr.vit_mrope_setup(inv_t, inv_h, inv_w, cu_d, grids_d, N, 2, c[0], c[1],
+                                            stream) for c in planes],
+           setup_bytes, N, "tokens", {"rotating_sets": len(planes)})
+    cos5, sin5 = planes[0]
+    qkr.vit_mrope_setup(inv_t, inv_h, inv_w, cu_d, grids_d, N, 2, cos5, sin5, stream)
+    del planes[1:]
     apply_bytes = 4 * N * 16 * 80 * 2 + 2 * N * 32 * 4 + 4 * 80 * 2
+    a5 = qkr.angle_table(cos5, sin5, W.SECTIONS_CONTIGUOUS, (16, 24, 24))
+    s5 = []
+    for _ in range(n_sets_for(apply_bytes)):
+        q5, k5 = w5.q.to(dev), w5.k.to(dev)
+        gq5, gk5 = w5.gamma_q.to(dev), w5.gamma_k.to(dev)
+        s5.append(([qkr.stream_desc(q5, k5, gq5, gk5)], torch.empty_like(q5),
+                   torch.empty_like(k5), (q5, k5, gq5, gk5)))
     record("fused_qk_norm_rope", "ViT apply N=%d H=16 D=80 rot=64 from the 3 planes" % N,
-           [lambda: qkr.fused_qk_norm_rope(d5, qo5, ko5, 64, 0, 1e-6, a5, 0, stream)],
-           apply_bytes, N, "tokens")
+           [lambda x=x: qkr.fused_qk_norm_rope(x[0], x[1], x[2], 64, 0, 1e-6, a5, 0, stream)
+            for x in s5], apply_bytes, N, "tokens", {"rotating_sets": len(s5)})
+    del s5, planes
 
     # config 2: RMSNorm + residual, decode rows and sweep points
     for R, hidden in [(1, 5120), (32, 5120), (1024, 8192), (4096, 8192), (16384, 8192),

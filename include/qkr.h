@@ -285,8 +285,10 @@ typedef struct qkr_launch_info {
     int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
     int32_t heads_per_item;  /* rope: head rows of one token a lane group loads
                                 together (pipelined kernel: head slots per CTA) */
-    int32_t pipelined;       /* rope: 1 if rows were staged by bulk copies into a
-                                shared-memory ring (warp-specialised kernel) */
+    int32_t pipelined;       /* rope: 0 rows loaded straight into registers (item
+                                kernel); 1 rows staged by bulk copies into a shared-
+                                memory ring (warp-specialised kernel); 2 rows streamed
+                                by every thread into a cp.async ring (streaming kernel) */
     int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
     int32_t block;           /* threads per CTA */
     int32_t direct_angles;   /* rope: 1 if each work item read its (cos, sin) straight
@@ -294,6 +296,8 @@ typedef struct qkr_launch_info {
                                 were staged per token in shared memory */
     int32_t overlap;         /* 1 if launched with programmatic stream serialisation
                                 (see qkr_launch_overlap) */
+    int32_t stages;          /* streaming kernel: passes in the row ring; else 0 */
+    int32_t reserved;        /* 0 */
     int64_t grid;            /* CTAs launched */
     int64_t launches;        /* kernel launches enqueued (0 for an empty call) */
 } qkr_launch_info;
@@ -310,14 +314,17 @@ qkr_status qkr_last_launch(qkr_launch_info *info);
 qkr_status qkr_launch_overlap(int32_t enable);
 
 /* Launch-shape override for the rope kernels, for tuning sweeps.  pipeline:
- * 0 automatic, 1 register kernel only, 2 bulk-copy pipelined kernel only
- * (calls it cannot serve then fail with QKR_ERR_CUDA); heads per work item
- * (1..4, register kernel) and tokens per CTA or per pipeline tile (1..64;
- * the staged-angle kernels cap it by their shared memory);
- * 0 keeps the automatic choice.  Process-wide.  Every shape computes
- * bit-identical results: a row's arithmetic does not depend on it.
- * Returns QKR_ERR_INVALID_ARG out of range. */
-qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta);
+ * 0 automatic, 1 item kernel (rows straight into registers), 2 bulk-copy
+ * pipelined kernel, 3 streaming kernel (cp.async row ring); calls a forced
+ * kernel cannot serve fail with QKR_ERR_CUDA.  heads per work item (1..4; the
+ * streaming kernel takes 1, 2 or 4), tokens per CTA or per pipeline tile
+ * (1..64; kernels that stage angles cap it by their shared memory) and ring
+ * depth of the streaming kernel (2..4); 0 keeps the automatic choice.
+ * Process-wide.  Every shape computes bit-identical results: a row's
+ * arithmetic does not depend on it.  Returns QKR_ERR_INVALID_ARG out of
+ * range. */
+qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,
+                         int32_t stages);
 
 /* Device status word of the library on the current device (0 = healthy).
  * Kernels that wait on shared-memory barriers give every wait a time budget;

@@ -63,6 +63,7 @@ class LaunchInfo(ctypes.Structure):
                 ("heads_per_item", ctypes.c_int32), ("pipelined", ctypes.c_int32),
                 ("cluster", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("direct_angles", ctypes.c_int32), ("overlap", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("grid", ctypes.c_int64), ("launches", ctypes.c_int64)]
 
 
@@ -83,7 +84,7 @@ def _load() -> ctypes.CDLL:
         "qkr_last_launch": [ctypes.POINTER(LaunchInfo)],
         "qkr_section_map": [V, I32, V, I64, V],
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
-        "qkr_tune_rope": [I32, I32, I32],
+        "qkr_tune_rope": [I32, I32, I32, I32],
         "qkr_launch_overlap": [I32],
         "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
     }
@@ -151,9 +152,11 @@ def _ptr_base(t, dtype, what):
     return t.untyped_storage().data_ptr(), t.storage_offset()
 
 
-def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 0) -> None:
-    """Override the rope kernels' launch shape (0 = automatic), for tuning."""
-    _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta))
+def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 0,
+              stages: int = 0) -> None:
+    """Override the rope kernels' launch shape (0 = automatic), for tuning.
+    pipeline: 1 item kernel, 2 bulk-copy pipelined kernel, 3 streaming kernel."""
+    _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta, stages))
 
 
 def launch_overlap(enable: bool) -> None:

@@ -351,6 +351,8 @@ qkr_status qkr_last_launch(qkr_launch_info *info)
     info->block = g_last.block;
     info->direct_angles = g_last.direct_angles;
     info->overlap = g_last.launches > 0 ? qkr::launch_overlap() : 0;
+    info->stages = g_last.stages;
+    info->reserved = 0;
     info->grid = g_last.grid;
     info->launches = g_last.launches;
     return QKR_OK;
@@ -365,13 +367,15 @@ qkr_status qkr_launch_overlap(int32_t enable)
     return QKR_OK;
 }
 
-qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta)
+qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,
+                         int32_t stages)
 {
-    if (pipeline < 0 || pipeline > 2 || heads_per_item < 0 || heads_per_item > 4 ||
-        tokens_per_cta < 0 || tokens_per_cta > 64)
+    if (pipeline < 0 || pipeline > 3 || heads_per_item < 0 || heads_per_item > 4 ||
+        tokens_per_cta < 0 || tokens_per_cta > 64 || stages < 0 || stages == 1 || stages > 4)
         return fail(QKR_ERR_INVALID_ARG,
-                    "pipeline in [0, 2], heads_per_item in [0, 4], tokens_per_cta in [0, 64]");
-    qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta);
+                    "pipeline in [0, 3], heads_per_item in [0, 4], tokens_per_cta in [0, 64], "
+                    "stages 0 or in [2, 4]");
+    qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta, stages);
     g_error.clear();
     return QKR_OK;
 }

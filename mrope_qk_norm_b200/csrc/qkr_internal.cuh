@@ -172,19 +172,21 @@ struct RopeParams {
     const float *sin;
     int64_t ld, plane_stride;
     int tab_vec4;             // table bases 16-byte aligned, ld and plane_stride % 4 == 0
+    int stages;               // streaming kernel: depth of the cp.async row ring
     int64_t token_offset;
 };
 
 struct LaunchRecord {
     int kernel = QKR_KERNEL_NONE;
     int lanes_per_row = 0, slots = 0, tokens_per_cta = 0, heads_per_item = 0, cluster = 1,
-        block = 0, pipelined = 0, direct_angles = 0;
+        block = 0, pipelined = 0, direct_angles = 0, stages = 0;
     int64_t grid = 0, launches = 0;
 };
 
 // Launch-shape override of the rope kernels (0: automatic); pipeline: 0 auto,
 // 1 register kernel only, 2 bulk-copy pipelined kernel only.
-void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta);
+void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta,
+                             int stages);
 
 // Bulk-copy pipelined rope kernel (rope_tma.cu); cudaErrorNotSupported when a
 // call is outside what it serves.

@@ -10,7 +10,7 @@
 #include <mutex>
 #include <vector>
 
-#include "rope_fast.cuh"
+#include "rope_stream.cuh"
 
 namespace qkr {
 namespace {
@@ -153,18 +153,19 @@ KernelFn pick_exchange(int lpr, int ns)
 #undef QKR_EXCHANGE_CASE
 }
 
-int g_force_pipe = 0;  // 0 automatic, 1 register kernel, 2 pipelined kernel
+int g_force_pipe = 0;  // 0 automatic, 1 item kernel, 2 bulk-copy kernel, 3 streaming kernel
 int g_force_u = 0;     // tuning override of heads per item (0: automatic)
 int g_force_tt = 0;    // tuning override of tokens per CTA (0: automatic)
+int g_force_s = 0;     // tuning override of the streaming ring depth (0: automatic)
 
-// CTAs of `fn` (256 threads, no dynamic shared memory) resident on the whole
-// current device at once.  Cached per (device, kernel): occupancy depends on
-// the kernel's registers only.
-cudaError_t resident_slots(KernelFn fn, int *slots)
+// CTAs of `fn` (256 threads, `smem` bytes of dynamic shared memory) resident
+// on the whole current device at once.  Cached per (device, kernel, smem).
+cudaError_t resident_slots(KernelFn fn, size_t smem, int *slots)
 {
     struct Entry {
         int dev;
         KernelFn fn;
+        size_t smem;
         int slots;
     };
     static std::mutex mu;
@@ -176,7 +177,7 @@ cudaError_t resident_slots(KernelFn fn, int *slots)
     {
         std::lock_guard<std::mutex> lock(mu);
         for (const Entry &c : cache)
-            if (c.dev == dev && c.fn == fn) {
+            if (c.dev == dev && c.fn == fn && c.smem == smem) {
                 *slots = c.slots;
                 return cudaSuccess;
             }
@@ -184,13 +185,89 @@ cudaError_t resident_slots(KernelFn fn, int *slots)
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
     if (e != cudaSuccess)
         return e;
     *slots = (per_sm > 0 ? per_sm : 1) * sms;
     std::lock_guard<std::mutex> lock(mu);
-    cache.push_back({dev, fn, *slots});
+    cache.push_back({dev, fn, smem, *slots});
     return cudaSuccess;
+}
+
+// Streaming kernel (rope_stream.cuh): heads per item U in {1, 2, 4}, ring
+// depth S, one wave of resident CTAs with at most kStreamTokens tokens each
+// (their staged angles share the CTA's shared memory with the ring).
+constexpr int kStreamTokens = 64;
+
+cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaStream_t stream,
+                               LaunchRecord *rec)
+{
+    // U = 2 heads per item with a two-pass ring was the best streaming shape
+    // in the sweeps (deeper rings and U = 4 cost resident CTAs).
+    int u = g_force_u > 0 ? g_force_u : 2;
+    if (u == 3)
+        u = 2;
+    const int S = g_force_s > 0 ? g_force_s : 2;
+    p.stages = S;
+    p.pw = layout == VECTOR ? p.D / 2 : p.P;
+    const int cs_ld = (p.pw + 3) & ~3;
+    const bool norm = p.norm != 0;
+    KernelFn fn = layout == PAIRED ? pick_stream_paired(lpr, ns, u, norm)
+                                   : pick_stream_vector(lpr, ns, u, norm);
+    if (!fn)
+        return cudaErrorInvalidConfiguration;
+    const size_t ring = (size_t)S * u * ns * kThreads * 16;
+    const size_t angles_max = (size_t)kStreamTokens * cs_ld * 2 * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(ring + angles_max));
+    if (e != cudaSuccess)
+        return e;
+    int64_t grid;
+    if (g_force_tt > 0) {
+        const int tt = g_force_tt < kStreamTokens ? g_force_tt : kStreamTokens;
+        grid = (p.T + tt - 1) / tt;
+    } else {
+        // One wave: the resident CTA count depends on the shared memory, which
+        // depends on the tokens per CTA, which depends on the grid; iterate
+        // from the largest reservation (each step can only shrink the
+        // per-CTA shared memory, so the wave stays resident).
+        const int64_t min_grid = (p.T + kStreamTokens - 1) / kStreamTokens;
+        int64_t tpc = kStreamTokens;
+        grid = min_grid;
+        for (int iter = 0; iter < 3; ++iter) {
+            int slots = 0;
+            e = resident_slots(fn, ring + (size_t)tpc * cs_ld * 2 * sizeof(float), &slots);
+            if (e != cudaSuccess)
+                return e;
+            int64_t g = p.T < slots ? p.T : slots;
+            if (g < min_grid)
+                g = min_grid;
+            if (g <= grid && iter > 0)
+                break;
+            grid = g;
+            tpc = (p.T + grid - 1) / grid;
+        }
+    }
+    if (grid < 1)
+        grid = 1;
+    p.tokens_per_cta = (int)((p.T + grid - 1) / grid);
+    const size_t smem = ring + (size_t)p.tokens_per_cta * cs_ld * 2 * sizeof(float);
+    e = launch(fn, dim3((unsigned)grid), dim3(kThreads), smem, stream, 1, p);
+    if (e == cudaSuccess && rec) {
+        *rec = LaunchRecord();
+        rec->kernel = layout == PAIRED ? QKR_KERNEL_ROPE_PAIRED : QKR_KERNEL_ROPE_VECTOR;
+        rec->lanes_per_row = lpr;
+        rec->slots = ns;
+        rec->tokens_per_cta = p.tokens_per_cta;
+        rec->heads_per_item = u;
+        rec->pipelined = 2;
+        rec->stages = S;
+        rec->cluster = 1;
+        rec->block = kThreads;
+        rec->grid = grid;
+        rec->launches = 1;
+    }
+    return e;
 }
 
 int pow2_ceil(int v)
@@ -203,11 +280,12 @@ int pow2_ceil(int v)
 
 }  // namespace
 
-void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta)
+void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta, int stages)
 {
     g_force_pipe = pipeline;
     g_force_u = heads_per_item;
     g_force_tt = tokens_per_cta;
+    g_force_s = stages;
 }
 
 cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t stream,
@@ -234,6 +312,16 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     // copy of the same bytes and the pipelined kernel is slower.
     if (layout != EXCHANGE && g_force_pipe == 2)
         return launch_rope_tma(p, layout == PAIRED, lpr, ns, g_force_tt, stream, rec);
+    if (p.T > INT_MAX)
+        return cudaErrorInvalidConfiguration;
+    // Angles from positions: the streaming kernel (sincosf once per token of a
+    // CTA's whole range, overlapped with the first row copies) measured ~4%
+    // faster than the item kernel's per-4-token staging on interleaved mRoPE
+    // (8192 x (16+8) heads); angles from a table: the item kernel with direct
+    // 16-byte table reads measured ~12% faster than the streaming kernel.
+    const bool stream_auto = g_force_pipe == 0 && p.angle_kind == QKR_ANGLE_POSITIONS;
+    if (layout != EXCHANGE && (g_force_pipe == 3 || stream_auto))
+        return launch_rope_stream(p, layout, lpr, ns, stream, rec);
     // staged (cos, sin) columns: GPT-J stages every pair of the head so pairs
     // past rot_dim rotate by the identity
     p.pw = layout == VECTOR ? p.D / 2 : p.P;
@@ -284,7 +372,7 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
         grid = (p.T + tt - 1) / tt;
     } else if (direct) {
         int slots = 0;
-        cudaError_t e = resident_slots(fn, &slots);
+        cudaError_t e = resident_slots(fn, 0, &slots);
         if (e != cudaSuccess)
             return e;
         grid = p.T < slots ? p.T : slots;

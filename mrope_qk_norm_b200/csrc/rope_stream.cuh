@@ -1,0 +1,344 @@
+// rope_stream.cuh -- the streaming variant of the item-based rope kernel.
+//
+// Same arithmetic as rope_fast.cuh (per-head RMSNorm of Q and K, text-first
+// concatenation, RoPE / mRoPE with packed fp32x2 math, one final rounding),
+// with the row traffic decoupled from the register file:
+//   * one wave of resident CTAs, each owning a balanced range of joint
+//     tokens;
+//   * every thread streams its own 16-byte row vectors into a shared-memory
+//     ring S passes ahead with cp.async (LDGSTS, L2-only), so about
+//     (S-1) x U x slots x 16 bytes per thread are in flight while it computes
+//     the current pass -- in the plain item kernel the loads of one pass only
+//     go out after the previous pass's math, and registers cap the depth;
+//   * a thread reads back only vectors it copied itself, so a pass needs no
+//     block barrier, only cp.async.wait_group on the thread's own groups;
+//   * the (cos, sin) of all of the CTA's tokens are staged once in shared
+//     memory at the start (sincosf of the fp32 position x inv_freq product,
+//     or the fp32 table), while the first passes' rows are already in
+//     flight.
+// Invalid vectors (past the head dim, past the item's heads, a dead item) are
+// zero-filled by the copy itself (source size 0), which keeps the sum of
+// squares exact.
+#pragma once
+
+#include "rope_fast.cuh"
+
+namespace qkr {
+
+// Exported by rope_stream_paired.cu / rope_stream_vector.cu.
+KernelFn pick_stream_paired(int lpr, int ns, int u, bool norm);
+KernelFn pick_stream_vector(int lpr, int ns, int u, bool norm);
+
+namespace {
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src, bool valid)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    const int src_size = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src),
+                 "r"(src_size)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+// Wait until at most `pending` of this thread's most recent groups are in
+// flight (the ring depth is a launch parameter; the instruction takes an
+// immediate).  This waits on the thread's own copies, which always complete.
+__device__ __forceinline__ void cp_async_wait(int pending)
+{
+    switch (pending) {
+    case 0: asm volatile("cp.async.wait_group 0;\n" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;\n" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;\n" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 3;\n" ::: "memory"); break;
+    }
+}
+
+// Shared-memory ring geometry: stage s, vector k = u * NS + slot, thread t
+// at ((s * U * NS + k) * kThreads + t) * 16 bytes -- a warp's accesses to one
+// vector index are 512 consecutive bytes (conflict-free 128-bit access).
+template <int U, int NS>
+__device__ __forceinline__ uint4 *ring_at(uint4 *ring, int stage, int k)
+{
+    return ring + ((size_t)(stage * U * NS + k) * kThreads + threadIdx.x);
+}
+
+template <int LAYOUT, int LPR, int NS, int U, bool NORM>
+__global__ void __launch_bounds__(kThreads)
+rope_stream_kernel(const __grid_constant__ RopeParams p)
+{
+    pdl_wait();
+    pdl_trigger();
+    constexpr int NQ = LAYOUT == PAIRED ? 4 : 2 * NS;
+    constexpr int NT = LAYOUT == PAIRED ? NS - 2 : 0;
+    constexpr int G = kThreads / LPR;
+    const int S = p.stages;
+    const bool ROUND = p.round_norm != 0;
+
+    extern __shared__ float4 smem[];
+    uint4 *ring = reinterpret_cast<uint4 *>(smem);
+    const int cs_ld = (p.pw + 3) & ~3;
+    float *cosv = reinterpret_cast<float *>(ring + (size_t)S * U * NS * kThreads);
+    float *sinv = cosv + p.tokens_per_cta * cs_ld;
+
+    const int64_t tok0 = (int64_t)blockIdx.x * p.T / gridDim.x;
+    const int ntok = (int)((int64_t)(blockIdx.x + 1) * p.T / gridDim.x - tok0);
+
+    const int lane = threadIdx.x % LPR;
+    const int grp = threadIdx.x / LPR;
+    const int D = p.D;
+    const int nvec = D >> 3;
+    const int npv = p.rot >> 4;
+    int vidx[NS];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+        int v;
+        if (LAYOUT == PAIRED)
+            v = k == 0 ? (lane < npv ? lane : -1)
+              : k == 1 ? (lane < npv ? lane + npv : -1)
+                       : 2 * npv + lane + LPR * (k - 2);
+        else
+            v = lane + LPR * k;
+        vidx[k] = (v >= 0 && v < nvec) ? v : -1;
+    }
+    int qpair[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+        qpair[q] = LAYOUT == PAIRED ? 8 * lane + 2 * q : 4 * (lane + LPR * (q >> 1)) + 2 * (q & 1);
+
+    const int nbq = (p.Hq + U - 1) / U;
+    const int gpt = nbq + (p.Hk + U - 1) / U;
+    const int items = ntok * gpt;
+    const int passes = (items + G - 1) / G;  // uniform across the CTA
+
+    // Copy this thread's vectors of pass `pass` into ring stage `pass % S`
+    // (one commit group per pass, empty past the last pass).
+    auto issue = [&](int pass) {
+        if (pass < passes) {
+            const Item m = decode_item<U>(p, tok0, pass * G + grp, items, gpt, nbq);
+            const int st = pass % S;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int k = 0; k < NS; ++k) {
+                    const bool ok = u < m.nh && vidx[k] >= 0;
+                    const __nv_bfloat16 *src = ok ? m.src + u * m.hs + 8 * vidx[k] : m.src;
+                    cp_async16(ring_at<U, NS>(ring, st, u * NS + k), src, ok);
+                }
+        }
+        cp_async_commit();
+    };
+
+    for (int s = 0; s < S - 1; ++s)
+        issue(s);
+    stage_angles(p, tok0, ntok, cs_ld, cosv, sinv);
+    __syncthreads();
+
+    for (int pass = 0; pass < passes; ++pass) {
+        issue(pass + S - 1);
+        cp_async_wait(S - 1);
+        const Item m = decode_item<U>(p, tok0, pass * G + grp, items, gpt, nbq);
+        const int st = pass % S;
+
+        float2 C[NQ], Sn[NQ];
+        {
+            const float *cr = cosv + m.tt * cs_ld;
+            const float *sr = sinv + m.tt * cs_ld;
+            const bool have = LAYOUT == PAIRED ? vidx[0] >= 0 : true;
+#pragma unroll
+            for (int q = 0; q < NQ; q += 2) {
+                const bool ok = have && (LAYOUT == PAIRED || vidx[q >> 1] >= 0);
+                const float4 c4 = ok ? *reinterpret_cast<const float4 *>(cr + qpair[q])
+                                     : make_float4(1.f, 1.f, 1.f, 1.f);
+                const float4 s4 = ok ? *reinterpret_cast<const float4 *>(sr + qpair[q])
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+                C[q] = f2(c4.x, c4.y);
+                C[q + 1] = f2(c4.z, c4.w);
+                Sn[q] = f2(s4.x, s4.y);
+                Sn[q + 1] = f2(s4.z, s4.w);
+            }
+        }
+        float2 GA[NQ], GB[NQ], GT[NT > 0 ? NT : 1][4];
+        if (NORM) {
+            const RopeStreamDev &Sd = m.s1 ? p.st[1] : p.st[0];
+            const __nv_bfloat16 *gam = m.isk ? Sd.gk : Sd.gq;
+            uint4 gv[NS];
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                if (LAYOUT == PAIRED) {
+                    const uint32_t wa = word(gv[0], q), wb = word(gv[1], q);
+                    GA[q] = f2(bf_lo(wa), bf_hi(wa));
+                    GB[q] = f2(bf_lo(wb), bf_hi(wb));
+                } else {
+                    const uint32_t w0 = word(gv[q >> 1], 2 * (q & 1));
+                    const uint32_t w1 = word(gv[q >> 1], 2 * (q & 1) + 1);
+                    GA[q] = f2(bf_lo(w0), bf_lo(w1));
+                    GB[q] = f2(bf_hi(w0), bf_hi(w1));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = word(gv[2 + k], i);
+                    GT[k][i] = f2(bf_lo(w), bf_hi(w));
+                }
+        }
+
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            uint4 raw[NS];
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                raw[k] = *ring_at<U, NS>(ring, st, u * NS + k);
+            float2 A[NQ], B[NQ], TL[NT > 0 ? NT : 1][4];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                if (LAYOUT == PAIRED) {
+                    const uint32_t wa = word(raw[0], q), wb = word(raw[1], q);
+                    A[q] = f2(bf_lo(wa), bf_hi(wa));
+                    B[q] = f2(bf_lo(wb), bf_hi(wb));
+                } else {
+                    const uint32_t w0 = word(raw[q >> 1], 2 * (q & 1));
+                    const uint32_t w1 = word(raw[q >> 1], 2 * (q & 1) + 1);
+                    A[q] = f2(bf_lo(w0), bf_lo(w1));
+                    B[q] = f2(bf_hi(w0), bf_hi(w1));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = word(raw[2 + k], i);
+                    TL[k][i] = f2(bf_lo(w), bf_hi(w));
+                }
+
+            if (NORM) {
+                float2 acc = f2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                    acc = __ffma2_rn(A[q], A[q], acc);
+                    acc = __ffma2_rn(B[q], B[q], acc);
+                }
+#pragma unroll
+                for (int k = 0; k < NT; ++k)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        acc = __ffma2_rn(TL[k][i], TL[k][i], acc);
+                float ss = acc.x + acc.y;
+#pragma unroll
+                for (int off = LPR / 2; off > 0; off >>= 1)
+                    ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
+                const float2 r2 = f2(r, r);
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                    A[q] = __fmul2_rn(__fmul2_rn(A[q], r2), GA[q]);
+                    B[q] = __fmul2_rn(__fmul2_rn(B[q], r2), GB[q]);
+                    if (ROUND) {
+                        A[q] = round2_bf16(A[q]);
+                        B[q] = round2_bf16(B[q]);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < NT; ++k)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        TL[k][i] = __fmul2_rn(__fmul2_rn(TL[k][i], r2), GT[k][i]);
+            }
+
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const float2 bs = __fmul2_rn(B[q], Sn[q]);
+                const float2 bc = __fmul2_rn(B[q], C[q]);
+                const float2 a2 = __ffma2_rn(A[q], C[q], f2(-bs.x, -bs.y));
+                const float2 b2 = __ffma2_rn(A[q], Sn[q], bc);
+                A[q] = a2;
+                B[q] = b2;
+            }
+
+            uint4 outv[NS];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                if (LAYOUT == PAIRED) {
+                    set_word(outv[0], q, pack2(A[q].x, A[q].y));
+                    set_word(outv[1], q, pack2(B[q].x, B[q].y));
+                } else {
+                    set_word(outv[q >> 1], 2 * (q & 1), pack2(A[q].x, B[q].x));
+                    set_word(outv[q >> 1], 2 * (q & 1) + 1, pack2(A[q].y, B[q].y));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < NT; ++k)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    set_word(outv[2 + k], i, pack2(TL[k][i].x, TL[k][i].y));
+
+            if (u < m.nh) {
+#pragma unroll
+                for (int k = 0; k < NS; ++k)
+                    if (vidx[k] >= 0)
+                        st_stream(m.dst + (int64_t)u * D + 8 * vidx[k], outv[k]);
+            }
+        }
+    }
+    cp_async_wait(0);  // nothing is left in flight (the trailing groups are empty)
+}
+
+template <int LAYOUT, int LPR, int NS, int U>
+KernelFn pick_stream_norm(bool norm)
+{
+    return norm ? rope_stream_kernel<LAYOUT, LPR, NS, U, true>
+                : rope_stream_kernel<LAYOUT, LPR, NS, U, false>;
+}
+
+template <int LAYOUT, int LPR, int NS>
+KernelFn pick_stream_u(int u, bool norm)
+{
+    switch (u) {
+    case 1: return pick_stream_norm<LAYOUT, LPR, NS, 1>(norm);
+    case 2: return pick_stream_norm<LAYOUT, LPR, NS, 2>(norm);
+    case 4: return pick_stream_norm<LAYOUT, LPR, NS, 4>(norm);
+    default: return nullptr;
+    }
+}
+
+template <int LAYOUT, int LPR>
+KernelFn pick_stream_ns(int ns, int u, bool norm)
+{
+    if constexpr (LAYOUT == PAIRED) {
+        switch (ns) {
+        case 2: return pick_stream_u<LAYOUT, LPR, 2>(u, norm);
+        case 3: return pick_stream_u<LAYOUT, LPR, 3>(u, norm);
+        case 4: return pick_stream_u<LAYOUT, LPR, 4>(u, norm);
+        default: return nullptr;
+        }
+    } else {
+        switch (ns) {
+        case 1: return pick_stream_u<LAYOUT, LPR, 1>(u, norm);
+        case 2: return pick_stream_u<LAYOUT, LPR, 2>(u, norm);
+        default: return nullptr;
+        }
+    }
+}
+
+template <int LAYOUT>
+KernelFn pick_stream(int lpr, int ns, int u, bool norm)
+{
+    switch (lpr) {
+    case 1: return pick_stream_ns<LAYOUT, 1>(ns, u, norm);
+    case 2: return pick_stream_ns<LAYOUT, 2>(ns, u, norm);
+    case 4: return pick_stream_ns<LAYOUT, 4>(ns, u, norm);
+    case 8: return pick_stream_ns<LAYOUT, 8>(ns, u, norm);
+    case 16: return pick_stream_ns<LAYOUT, 16>(ns, u, norm);
+    default: return nullptr;
+    }
+}
+
+}  // namespace
+}  // namespace qkr

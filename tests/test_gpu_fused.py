@@ -386,3 +386,61 @@ def test_one_wave_grid_covers_every_token():
         assert rec["direct_angles"] == 1
         assert rec["grid"] <= w.n_tokens
         assert rec["tokens_per_cta"] == -(-w.n_tokens // rec["grid"])
+
+
+def _with_shape(w, pipe, u=0, tt=0, stages=0, flags=0):
+    try:
+        qkr.tune_rope(pipe, u, tt, stages)
+        out = run_fused(w, flags)
+        rec = qkr.last_launch()
+    finally:
+        qkr.tune_rope(0, 0, 0, 0)
+    return out, rec
+
+
+def _stream_cases():
+    cases = []
+    for D, rot, pairing in [(128, 128, W.PAIRING_GPTJ), (128, 128, W.PAIRING_NEOX),
+                            (80, 64, W.PAIRING_NEOX), (256, 128, W.PAIRING_NEOX),
+                            (64, 22, W.PAIRING_GPTJ), (32, 16, W.PAIRING_NEOX),
+                            (128, 0, W.PAIRING_NEOX)]:
+        pos = np.random.default_rng(D + 7 * rot).integers(0, 50000, (1, 61)).astype(np.int32)
+        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                          inv_freq=W.inv_freq(1e4, max(rot // 2, 1), max(rot, 2)).numpy())
+        cases.append(("pos D=%d rot=%d p=%d" % (D, rot, pairing),
+                      W.random_rope_case(D * 3 + rot, [61], 7, 3, D, rot, pairing, A)))
+    cases.append(("joint gptj table", W.config3(seed=101, T_txt=37, img_h=9, img_w=11, H=12,
+                                                 D=128, pairing=W.PAIRING_GPTJ)))
+    return cases
+
+
+@pytest.mark.parametrize("name,w", _stream_cases(), ids=lambda v: v if isinstance(v, str) else "")
+def test_streaming_kernel_equals_item_kernel(name, w):
+    """The cp.async streaming kernel computes the same bits as the item kernel,
+    for every layout, with positions and tables, and matches the oracle."""
+    (qa, ka), ra = _with_shape(w, 3)
+    (qb, kb), rb = _with_shape(w, 1)
+    assert ra["pipelined"] == 2 and ra["stages"] >= 2 and rb["pipelined"] == 0
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16)), name
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16)), name
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle,
+                                 norm=w.norm)
+    assert_bf16_close(qa, rq, name + " q")
+    assert_bf16_close(ka, rk, name + " k")
+
+
+def test_streaming_kernel_shapes_and_round_flag():
+    """Heads per item, ring depth and token split do not change a bit; the
+    bf16-rounded-normalised contract is served too."""
+    w = W.config3(seed=103, T_txt=45, img_h=7, img_w=13, H=10, D=128, pairing=W.PAIRING_NEOX)
+    ref, _ = _with_shape(w, 1)
+    for u, tt, st in [(1, 0, 2), (2, 1, 3), (4, 7, 4), (4, 64, 2), (2, 0, 4)]:
+        out, rec = _with_shape(w, 3, u, tt, st)
+        assert rec["heads_per_item"] == u and rec["stages"] == st
+        assert torch.equal(out[0].view(torch.int16), ref[0].view(torch.int16)), (u, tt, st)
+        assert torch.equal(out[1].view(torch.int16), ref[1].view(torch.int16)), (u, tt, st)
+    flags = qkr.FLAG_ROUND_NORMALIZED_BF16
+    (qa, ka), _ = _with_shape(w, 3, flags=flags)
+    (qb, kb), _ = _with_shape(w, 1, flags=flags)
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
