@@ -195,8 +195,8 @@ cudaError_t resident_slots(KernelFn fn, size_t smem, int *slots)
 }
 
 // Streaming kernel (rope_stream.cuh): heads per item U in {1, 2, 4}, ring
-// depth S, one wave of resident CTAs with at most kStreamTokens tokens each
-// (their staged angles share the CTA's shared memory with the ring).
+// depth S, at most kStreamTokens tokens per CTA (their staged angles share
+// the CTA's shared memory with the ring).
 constexpr int kStreamTokens = 64;
 
 cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaStream_t stream,
@@ -222,32 +222,23 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
                                          (int)(ring + angles_max));
     if (e != cudaSuccess)
         return e;
+    // Token split: 8 tokens per CTA once that still gives four waves of
+    // resident CTAs, else 4.  On interleaved mRoPE (8192 x (16+8) heads,
+    // whole and chunked at 2457) this was within 3% of the best fixed split
+    // in each case; a single wave of larger ranges was 3-15% slower (each
+    // CTA's staging prologue is exposed once per range).
     int64_t grid;
-    if (g_force_tt > 0) {
-        const int tt = g_force_tt < kStreamTokens ? g_force_tt : kStreamTokens;
-        grid = (p.T + tt - 1) / tt;
-    } else {
-        // One wave: the resident CTA count depends on the shared memory, which
-        // depends on the tokens per CTA, which depends on the grid; iterate
-        // from the largest reservation (each step can only shrink the
-        // per-CTA shared memory, so the wave stays resident).
-        const int64_t min_grid = (p.T + kStreamTokens - 1) / kStreamTokens;
-        int64_t tpc = kStreamTokens;
-        grid = min_grid;
-        for (int iter = 0; iter < 3; ++iter) {
-            int slots = 0;
-            e = resident_slots(fn, ring + (size_t)tpc * cs_ld * 2 * sizeof(float), &slots);
-            if (e != cudaSuccess)
-                return e;
-            int64_t g = p.T < slots ? p.T : slots;
-            if (g < min_grid)
-                g = min_grid;
-            if (g <= grid && iter > 0)
-                break;
-            grid = g;
-            tpc = (p.T + grid - 1) / grid;
-        }
+    int tt = g_force_tt;
+    if (tt <= 0) {
+        int slots = 0;
+        e = resident_slots(fn, ring + (size_t)8 * cs_ld * 2 * sizeof(float), &slots);
+        if (e != cudaSuccess)
+            return e;
+        tt = p.T >= 4 * (int64_t)slots ? 8 : 4;
     }
+    if (tt > kStreamTokens)
+        tt = kStreamTokens;
+    grid = (p.T + tt - 1) / tt;
     if (grid < 1)
         grid = 1;
     p.tokens_per_cta = (int)((p.T + grid - 1) / grid);

@@ -3,8 +3,7 @@
 // Same arithmetic as rope_fast.cuh (per-head RMSNorm of Q and K, text-first
 // concatenation, RoPE / mRoPE with packed fp32x2 math, one final rounding),
 // with the row traffic decoupled from the register file:
-//   * one wave of resident CTAs, each owning a balanced range of joint
-//     tokens;
+//   * CTAs each owning a balanced range of a few joint tokens (4-8);
 //   * every thread streams its own 16-byte row vectors into a shared-memory
 //     ring S passes ahead with cp.async (LDGSTS, L2-only), so about
 //     (S-1) x U x slots x 16 bytes per thread are in flight while it computes
