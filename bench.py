@@ -295,6 +295,28 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
            [lambda s=s: s.launch(stream) for s in sets], b3, 4608, "tokens")
     del sets
 
+    # config 3 as the joint Q/K/V op: V of both streams copied into the joint V
+    w3 = W.config3()
+    b3v = b3 + 2 * 4608 * 24 * 128 * 2
+    qkv_sets = []
+    for i in range(n_sets_for(b3v)):
+        fs = FusedSet(w3, dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(3000 + i)
+        vs = [torch.randn(s[0].shape, device=dev, generator=g).to(torch.bfloat16)
+              for s in fs.streams]
+        descs = [qkr.stream_desc(s[0], s[1], s[2], s[3], v) for s, v in zip(fs.streams, vs)]
+        vo = torch.empty(4608, 24, 128, dtype=torch.bfloat16, device=dev)
+        qkv_sets.append((fs, descs, vo, vs))
+
+    def qkv(x):
+        fs, descs, vo, _ = x
+        qkr.fused_qkv_norm_rope(descs, fs.qo, fs.ko, vo, 128, w3.pairing, w3.eps, fs.angle,
+                                0, stream)
+    record("fused_qkv_norm_rope", "joint Q/K/V 512+4096 tokens H=24 D=128 GPT-J",
+           [lambda x=x: qkv(x) for x in qkv_sets], b3v, 4608, "tokens")
+    del qkv_sets
+
     # config 4: interleaved mRoPE (no norm), unchunked and chunked at 2457
     w4 = W.config4()
     T, Hq, Hkv, D = 8192, 16, 8, 128

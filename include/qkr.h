@@ -5,6 +5,8 @@
  *
  *   fused_qk_norm_rope  per-head RMSNorm of Q and K, optional text/image
  *                       concatenation, RoPE (NeoX or GPT-J pairing), one launch.
+ *   fused_qkv_norm_rope the same, with V concatenated (copied unchanged)
+ *                       into a joint V output in the same launch.
  *   mrope_apply         multi-section RoPE (contiguous or interleaved
  *                       sections) with a token offset for chunked launches,
  *                       optional per-head RMSNorm.
@@ -103,11 +105,13 @@ enum {
     QKR_FLAG_ROUND_NORMALIZED_BF16 = 1u
 };
 
-/* One input stream of fused_qk_norm_rope.  q and k are bf16 device pointers;
- * element (t, h, d) of Q is at q + q_offset + t*q_tok_stride +
- * h*q_head_stride + d (d contiguous), likewise K.  Offsets may exceed 2^31
- * elements: all address arithmetic is 64-bit (vllm-omni #7600, 64-bit row
- * addressing for large storage offsets).  gamma_q / gamma_k: bf16 [D] device. */
+/* One input stream of fused_qk_norm_rope / fused_qkv_norm_rope.  q, k and v
+ * are bf16 device pointers; element (t, h, d) of Q is at q + q_offset +
+ * t*q_tok_stride + h*q_head_stride + d (d contiguous), likewise K and V.
+ * Offsets may exceed 2^31 elements: all address arithmetic is 64-bit
+ * (vllm-omni #7600, 64-bit row addressing for large storage offsets).
+ * gamma_q / gamma_k: bf16 [D] device.  The v fields are read only by
+ * fused_qkv_norm_rope (zero them otherwise). */
 typedef struct qkr_stream_desc {
     const void *q;
     const void *k;
@@ -120,6 +124,10 @@ typedef struct qkr_stream_desc {
     int64_t n_tokens;
     const void *gamma_q;
     const void *gamma_k;
+    const void *v;
+    int64_t v_offset;
+    int64_t v_tok_stride;
+    int64_t v_head_stride;
 } qkr_stream_desc;
 
 /* Angle source (see QKR_ANGLE_*).  Unused fields are ignored.
@@ -177,6 +185,27 @@ qkr_status fused_qk_norm_rope(void *stream, const qkr_stream_desc *streams, int3
                               int64_t k_out_tok_stride, int64_t Hq, int64_t Hk, int64_t D,
                               int64_t rot_dim, int32_t pairing, float eps,
                               const qkr_angle_desc *angle, uint32_t flags);
+
+/*
+ * fused_qkv_norm_rope -- the joint Q/K/V form of the same op (vllm-omni #7600,
+ * Purpose: the fused joint op takes Q, K and V as zero-copy strided views and
+ * writes the concatenated joint Q, K and V in one launch).  Q and K exactly as
+ * fused_qk_norm_rope; each stream's V rows are copied bit for bit, text first,
+ * into v_out, with no norm and no rotation.
+ *
+ *   v_out            bf16 device [T0+T1, Hv, D]; row n starts at
+ *                    v_out + n*v_out_tok_stride (heads dense).  Fresh: must
+ *                    not overlap any input or the other outputs.
+ *   Hv               V heads per token, >= 1 (V shares D with Q and K).
+ * Every stream with tokens needs v (and its strides, same rules as q / k).
+ * Errors, alignment and the remaining arguments as fused_qk_norm_rope.
+ */
+qkr_status fused_qkv_norm_rope(void *stream, const qkr_stream_desc *streams, int32_t n_streams,
+                               void *q_out, void *k_out, void *v_out, int64_t q_out_tok_stride,
+                               int64_t k_out_tok_stride, int64_t v_out_tok_stride, int64_t Hq,
+                               int64_t Hk, int64_t Hv, int64_t D, int64_t rot_dim,
+                               int32_t pairing, float eps, const qkr_angle_desc *angle,
+                               uint32_t flags);
 
 /*
  * mrope_apply -- multi-section RoPE (llama.cpp fork #286, "The change":

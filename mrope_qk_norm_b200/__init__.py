@@ -27,7 +27,7 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
                 4: "vit_setup", 5: "rms_rows", 6: "rms_cluster", 7: "section_map",
                 8: "vit_positions"}
 
-EXPORTS = ("fused_qk_norm_rope", "mrope_apply", "vit_mrope_setup", "rms_norm_residual",
+EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "vit_mrope_setup", "rms_norm_residual",
            "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
            "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status", "qkr_launch_overlap")
 
@@ -44,7 +44,9 @@ class StreamDesc(ctypes.Structure):
                 ("q_tok_stride", ctypes.c_int64), ("q_head_stride", ctypes.c_int64),
                 ("k_tok_stride", ctypes.c_int64), ("k_head_stride", ctypes.c_int64),
                 ("n_tokens", ctypes.c_int64),
-                ("gamma_q", ctypes.c_void_p), ("gamma_k", ctypes.c_void_p)]
+                ("gamma_q", ctypes.c_void_p), ("gamma_k", ctypes.c_void_p),
+                ("v", ctypes.c_void_p), ("v_offset", ctypes.c_int64),
+                ("v_tok_stride", ctypes.c_int64), ("v_head_stride", ctypes.c_int64)]
 
 
 class AngleDesc(ctypes.Structure):
@@ -77,6 +79,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "fused_qk_norm_rope": [V, ctypes.POINTER(StreamDesc), I32, V, V, I64, I64, I64, I64, I64,
                                I64, I32, F, ctypes.POINTER(AngleDesc), U32],
+        "fused_qkv_norm_rope": [V, ctypes.POINTER(StreamDesc), I32, V, V, V, I64, I64, I64, I64,
+                                I64, I64, I64, I64, I32, F, ctypes.POINTER(AngleDesc), U32],
         "mrope_apply": [V, V, V, V, V, I64, I64, I64, I64, I64, I64, I64, I64, I64, V, I64, I64,
                         I64, V, V, I32, I32, V, V, F, U32],
         "vit_mrope_setup": [V, V, V, V, I64, I64, I64, V, V, I64, I64, I64, V, V],
@@ -183,8 +187,9 @@ def last_launch() -> dict:
 # fused_qk_norm_rope
 # --------------------------------------------------------------------------
 
-def stream_desc(q, k, gamma_q, gamma_k) -> StreamDesc:
-    """Descriptor for a [T, H, D] Q/K view (any token/head strides, D dense)."""
+def stream_desc(q, k, gamma_q, gamma_k, v=None) -> StreamDesc:
+    """Descriptor for [T, H, D] Q/K (and optionally V) views (any token/head
+    strides, D dense)."""
     bf = torch.bfloat16
     if q.dim() != 3 or k.dim() != 3 or q.shape[0] != k.shape[0]:
         raise ValueError("q and k must be [T, H, D] views with the same T")
@@ -198,7 +203,12 @@ def stream_desc(q, k, gamma_q, gamma_k) -> StreamDesc:
     d.n_tokens = q.shape[0]
     d.gamma_q = _ptr(gamma_q, bf, "gamma_q")
     d.gamma_k = _ptr(gamma_k, bf, "gamma_k")
-    d._keep = (q, k, gamma_q, gamma_k)  # the descriptor holds raw pointers into these
+    if v is not None:
+        if v.dim() != 3 or v.shape[0] != q.shape[0] or v.stride(2) != 1:
+            raise ValueError("v must be a [T, Hv, D] view with the same T and a contiguous D")
+        d.v, d.v_offset = _ptr_base(v, bf, "v")
+        d.v_tok_stride, d.v_head_stride = v.stride(0), v.stride(1)
+    d._keep = (q, k, gamma_q, gamma_k, v)  # the descriptor holds raw pointers into these
     return d
 
 
@@ -260,6 +270,23 @@ def fused_qk_norm_rope(streams, q_out, k_out, rot_dim, pairing, eps, angle: Angl
         _ptr(k_out, torch.bfloat16, "k_out"), q_out.stride(0), k_out.stride(0),
         q_out.shape[1], k_out.shape[1], q_out.shape[2], rot_dim, pairing, eps,
         ctypes.byref(angle), flags))
+
+
+def fused_qkv_norm_rope(streams, q_out, k_out, v_out, rot_dim, pairing, eps,
+                        angle: AngleDesc, flags=0, stream=None):
+    """streams: list of (q, k, gamma_q, gamma_k, v) tuples or StreamDesc objects
+    with v set.  q_out / k_out / v_out: [T_total, H, D] bf16 (heads dense); V
+    rows are copied unchanged, text first."""
+    descs = [s if isinstance(s, StreamDesc) else stream_desc(*s) for s in streams]
+    arr = (StreamDesc * len(descs))(*descs)
+    for name, t in (("q_out", q_out), ("k_out", k_out), ("v_out", v_out)):
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("%s must be [T, H, D] with dense heads" % name)
+    _check(_lib.fused_qkv_norm_rope(
+        _stream(stream), arr, len(descs), _ptr(q_out, torch.bfloat16, "q_out"),
+        _ptr(k_out, torch.bfloat16, "k_out"), _ptr(v_out, torch.bfloat16, "v_out"),
+        q_out.stride(0), k_out.stride(0), v_out.stride(0), q_out.shape[1], k_out.shape[1],
+        v_out.shape[1], q_out.shape[2], rot_dim, pairing, eps, ctypes.byref(angle), flags))
 
 
 # --------------------------------------------------------------------------

@@ -187,16 +187,20 @@ qkr_status check_geometry(int64_t Hq, int64_t Hk, int64_t D, int64_t rot, int32_
     return QKR_OK;
 }
 
-// Shared body of fused_qk_norm_rope and mrope_apply.  `inplace_ok` admits
-// outputs equal to the inputs with identical strides (mrope_apply).
+// Shared body of fused_qk_norm_rope, fused_qkv_norm_rope and mrope_apply.
+// `inplace_ok` admits outputs equal to the inputs with identical strides
+// (mrope_apply).  Hv > 0 routes each stream's V rows into v_out unchanged.
 qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_streams,
                      void *q_out, void *k_out, int64_t qo_ts, int64_t ko_ts, int64_t Hq,
                      int64_t Hk, int64_t D, int64_t rot, int32_t pairing, float eps,
-                     const qkr_angle_desc *angle, uint32_t flags, bool norm, bool inplace_ok)
+                     const qkr_angle_desc *angle, uint32_t flags, bool norm, bool inplace_ok,
+                     int64_t Hv = 0, void *v_out = nullptr, int64_t vo_ts = 0)
 {
     qkr_status st = check_geometry(Hq, Hk, D, rot, pairing, eps);
     if (st != QKR_OK)
         return st;
+    if (Hv < 0 || Hq + Hk + Hv > 65536)
+        return fail(QKR_ERR_INVALID_ARG, "V head count out of range");
     if (!streams || n_streams < 1 || n_streams > 2)
         return fail(QKR_ERR_INVALID_ARG, "need 1 or 2 stream descriptors");
     if (flags & ~(uint32_t)QKR_FLAG_ROUND_NORMALIZED_BF16)
@@ -219,10 +223,20 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     if (qo_ts < Hq * D || ko_ts < Hk * D || qo_ts % 8 || ko_ts % 8)
         return fail(QKR_ERR_UNSUPPORTED,
                     "output token strides must be multiples of 8 and hold a token's heads");
+    if (Hv > 0) {
+        if (!v_out)
+            return fail(QKR_ERR_INVALID_ARG, "v_out must be non-NULL");
+        if (!aligned16(v_out))
+            return fail(QKR_ERR_UNSUPPORTED, "v_out must be 16-byte aligned");
+        if (vo_ts < Hv * D || vo_ts % 8)
+            return fail(QKR_ERR_UNSUPPORTED,
+                        "v_out token stride must be a multiple of 8 and hold a token's heads");
+    }
 
     qkr::RopeParams p = {};
     int64_t T = 0;
-    const __nv_bfloat16 *qb[2] = {nullptr, nullptr}, *kb[2] = {nullptr, nullptr};
+    const __nv_bfloat16 *qb[2] = {nullptr, nullptr}, *kb[2] = {nullptr, nullptr},
+                        *vb[2] = {nullptr, nullptr};
     for (int s = 0; s < n_streams; ++s) {
         const qkr_stream_desc &d = streams[s];
         if (d.n_tokens < 0)
@@ -268,6 +282,28 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
         p.st[s].k_hs = d.k_head_stride;
         p.st[s].gq = static_cast<const __nv_bfloat16 *>(d.gamma_q);
         p.st[s].gk = static_cast<const __nv_bfloat16 *>(d.gamma_k);
+        if (Hv > 0) {
+            if (!d.v)
+                return fail(QKR_ERR_INVALID_ARG, "stream %d: v must be non-NULL", s);
+            if (d.v_offset < 0 || d.v_offset > ((int64_t)1 << 60))
+                return fail(QKR_ERR_INVALID_ARG, "stream %d: v storage offset out of range", s);
+            if (d.v_tok_stride <= 0 || d.v_head_stride < D)
+                return fail(QKR_ERR_UNSUPPORTED,
+                            "stream %d: v strides must be positive and heads must not overlap",
+                            s);
+            if (d.v_tok_stride % 8 || d.v_head_stride % 8 || d.v_offset % 8)
+                return fail(QKR_ERR_UNSUPPORTED,
+                            "stream %d: v offset and strides must be multiples of 8 elements", s);
+            if (!view_fits(d.n_tokens, d.v_tok_stride, Hv, d.v_head_stride, D))
+                return fail(QKR_ERR_INVALID_ARG, "stream %d: v view exceeds the address range",
+                            s);
+            vb[s] = static_cast<const __nv_bfloat16 *>(d.v) + d.v_offset;
+            if (!aligned16(vb[s]))
+                return fail(QKR_ERR_UNSUPPORTED, "stream %d: v must be 16-byte aligned", s);
+            p.st[s].v = vb[s];
+            p.st[s].v_ts = d.v_tok_stride;
+            p.st[s].v_hs = d.v_head_stride;
+        }
         T += d.n_tokens;
     }
     if (T > ((int64_t)1 << 40))
@@ -280,6 +316,14 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     const Span so_k = view_span(k_out, T, ko_ts, Hk, D, D);
     if (overlap(so_q, so_k))
         return fail(QKR_ERR_UNSUPPORTED, "q_out and k_out overlap");
+    Span so_v;
+    if (Hv > 0) {
+        if (!view_fits(T, vo_ts, 1, 0, Hv * D))
+            return fail(QKR_ERR_INVALID_ARG, "v_out view exceeds the address range");
+        so_v = view_span(v_out, T, vo_ts, Hv, D, D);
+        if (overlap(so_v, so_q) || overlap(so_v, so_k))
+            return fail(QKR_ERR_UNSUPPORTED, "v_out overlaps q_out or k_out");
+    }
     for (int s = 0; s < n_streams; ++s) {
         const qkr_stream_desc &d = streams[s];
         if (d.n_tokens == 0)
@@ -295,6 +339,14 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
             return fail(QKR_ERR_UNSUPPORTED,
                         inplace_ok ? "outputs overlap inputs (only exact in-place is allowed)"
                                    : "outputs must not overlap the inputs (fresh outputs)");
+        if (Hv > 0) {
+            const Span si_v =
+                view_span(vb[s], d.n_tokens, d.v_tok_stride, Hv, d.v_head_stride, D);
+            if (overlap(so_v, si_q) || overlap(so_v, si_k) || overlap(so_v, si_v) ||
+                overlap(so_q, si_v) || overlap(so_k, si_v))
+                return fail(QKR_ERR_UNSUPPORTED,
+                            "outputs must not overlap the inputs (fresh outputs)");
+        }
     }
 
     const int64_t P = rot / 2;
@@ -307,15 +359,18 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
         p.split = 0;
     p.q_out = static_cast<__nv_bfloat16 *>(q_out);
     p.k_out = static_cast<__nv_bfloat16 *>(k_out);
+    p.v_out = static_cast<__nv_bfloat16 *>(v_out);
     p.qo_ts = qo_ts;
     p.ko_ts = ko_ts;
+    p.vo_ts = vo_ts;
+    p.Hv = (int)Hv;
     p.T = T;
     p.Hq = (int)Hq;
     p.Hk = (int)Hk;
     p.D = (int)D;
     p.rot = (int)rot;
     p.P = (int)P;
-    p.rows_per_token = (int)(Hq + Hk);
+    p.rows_per_token = (int)(Hq + Hk + Hv);
     p.eps = eps;
     p.inv_D = 1.0f / (float)D;
     p.norm = norm ? 1 : 0;
@@ -399,6 +454,20 @@ qkr_status fused_qk_norm_rope(void *stream, const qkr_stream_desc *streams, int3
     return rope_call(stream, streams, n_streams, q_out, k_out, q_out_tok_stride,
                      k_out_tok_stride, Hq, Hk, D, rot_dim, pairing, eps, angle, flags,
                      /*norm=*/true, /*inplace_ok=*/false);
+}
+
+qkr_status fused_qkv_norm_rope(void *stream, const qkr_stream_desc *streams, int32_t n_streams,
+                               void *q_out, void *k_out, void *v_out, int64_t q_out_tok_stride,
+                               int64_t k_out_tok_stride, int64_t v_out_tok_stride, int64_t Hq,
+                               int64_t Hk, int64_t Hv, int64_t D, int64_t rot_dim,
+                               int32_t pairing, float eps, const qkr_angle_desc *angle,
+                               uint32_t flags)
+{
+    if (Hv < 1)
+        return fail(QKR_ERR_INVALID_ARG, "Hv must be >= 1 (use fused_qk_norm_rope without V)");
+    return rope_call(stream, streams, n_streams, q_out, k_out, q_out_tok_stride,
+                     k_out_tok_stride, Hq, Hk, D, rot_dim, pairing, eps, angle, flags,
+                     /*norm=*/true, /*inplace_ok=*/false, Hv, v_out, v_out_tok_stride);
 }
 
 qkr_status mrope_apply(void *stream, const void *q, const void *k, void *q_out, void *k_out,

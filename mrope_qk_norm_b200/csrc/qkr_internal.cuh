@@ -144,7 +144,8 @@ __device__ __forceinline__ int section_axis(int mode, const int (&sec)[4], int j
 struct RopeStreamDev {
     const __nv_bfloat16 *q;   // already advanced by the storage offset
     const __nv_bfloat16 *k;
-    int64_t q_ts, q_hs, k_ts, k_hs;
+    const __nv_bfloat16 *v;   // joint Q/K/V only (copied unchanged)
+    int64_t q_ts, q_hs, k_ts, k_hs, v_ts, v_hs;
     const __nv_bfloat16 *gq;
     const __nv_bfloat16 *gk;
 };
@@ -154,10 +155,12 @@ struct RopeParams {
     int64_t split;            // joint row where stream 1 starts (INT64_MAX: one stream)
     __nv_bfloat16 *q_out;
     __nv_bfloat16 *k_out;
-    int64_t qo_ts, ko_ts;
+    __nv_bfloat16 *v_out;     // joint Q/K/V only
+    int64_t qo_ts, ko_ts, vo_ts;
     int64_t T;                // joint tokens in this launch
     int Hq, Hk, D, rot, P;
-    int rows_per_token;       // Hq + Hk
+    int Hv;                   // V heads copied into v_out (0: Q/K only)
+    int rows_per_token;       // Hq + Hk + Hv
     int tokens_per_cta;
     int pw;                   // (cos, sin) columns staged per token: P, or D/2 for GPT-J
                               // (pairs in [P, D/2) get the identity (1, 0))

@@ -156,14 +156,53 @@ __device__ __forceinline__ Item decode_item(const RopeParams &p, int64_t tok0, i
     const int64_t n = tok0 + r.tt;
     r.s1 = n >= p.split;
     const int64_t t = r.s1 ? n - p.split : n;
-    const RopeStreamDev &S0 = p.st[0];
-    const RopeStreamDev &S1 = p.st[1];
-    const __nv_bfloat16 *base = r.isk ? (r.s1 ? S1.k : S0.k) : (r.s1 ? S1.q : S0.q);
-    const int64_t ts = r.isk ? (r.s1 ? S1.k_ts : S0.k_ts) : (r.s1 ? S1.q_ts : S0.q_ts);
-    r.hs = r.isk ? (r.s1 ? S1.k_hs : S0.k_hs) : (r.s1 ? S1.q_hs : S0.q_hs);
+    const RopeStreamDev &S = r.s1 ? p.st[1] : p.st[0];
+    const __nv_bfloat16 *base = r.isk ? S.k : S.q;
+    const int64_t ts = r.isk ? S.k_ts : S.q_ts;
+    r.hs = r.isk ? S.k_hs : S.q_hs;
     r.src = base + t * ts + (int64_t)h0 * r.hs;
     r.dst = (r.isk ? p.k_out : p.q_out) + n * (r.isk ? p.ko_ts : p.qo_ts) + (int64_t)h0 * p.D;
     return r;
+}
+
+// Joint Q/K/V: after its Q/K items a CTA copies the V rows of its tokens into
+// v_out unchanged, two rows per group at a time, with the lanes' own vector
+// slots (which cover the whole head dim in both layouts).  No math and no
+// shuffles, and a small register footprint, so the Q/K loop keeps its
+// occupancy.
+template <int NS, int LPR>
+__device__ __forceinline__ void copy_v_rows(const RopeParams &p, int64_t tok0, int ntok,
+                                            const int (&vidx)[NS])
+{
+    constexpr int G = kThreads / LPR;
+    const int rows = ntok * p.Hv;
+    for (int r0 = threadIdx.x / LPR; r0 < rows; r0 += 2 * G) {
+        uint4 raw[2][NS];
+        __nv_bfloat16 *dst[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int r = r0 + j * G;
+            const bool live = r < rows;
+            const int tt = live ? r / p.Hv : 0;
+            const int h = live ? r - tt * p.Hv : 0;
+            const int64_t n = tok0 + tt;
+            const bool s1 = n >= p.split;
+            const int64_t t = s1 ? n - p.split : n;
+            const RopeStreamDev &S = s1 ? p.st[1] : p.st[0];
+            const __nv_bfloat16 *src = S.v + t * S.v_ts + (int64_t)h * S.v_hs;
+            dst[j] = live ? p.v_out + n * p.vo_ts + (int64_t)h * p.D : nullptr;
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                raw[j][k] = (live && vidx[k] >= 0) ? ld_stream(src + 8 * vidx[k])
+                                                   : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                if (dst[j] && vidx[k] >= 0)
+                    st_stream(dst[j] + 8 * vidx[k], raw[j][k]);
+    }
 }
 
 template <int LAYOUT, int LPR, int NS, int U, bool NORM, bool ROUND, bool DIRECT>
@@ -215,6 +254,10 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
         qpair[q] = LAYOUT == PAIRED ? 8 * lane + 2 * q : 4 * (lane + LPR * (q >> 1)) + 2 * (q & 1);
+
+    // joint Q/K/V: the CTA's V rows first (plain copies), then its Q/K items
+    if (p.Hv > 0)
+        copy_v_rows<NS, LPR>(p, tok0, ntok, vidx);
 
     const int nbq = (p.Hq + U - 1) / U;
     const int gpt = nbq + (p.Hk + U - 1) / U;

@@ -60,20 +60,25 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
         const int64_t n = tok0 + tt;
         const bool s1 = n >= p.split;
         const int64_t t = s1 ? n - p.split : n;
-        const bool isk = h >= p.Hq;
-        const int hh = isk ? h - p.Hq : h;
+        // rows of a token: Hq Q heads, Hk K heads, then Hv V heads (copied)
+        const bool isv = h >= p.Hq + p.Hk;
+        const bool isk = !isv && h >= p.Hq;
+        const int hh = isv ? h - p.Hq - p.Hk : isk ? h - p.Hq : h;
         const RopeStreamDev &S = s1 ? p.st[1] : p.st[0];
-        const __nv_bfloat16 *src = (isk ? S.k : S.q) + t * (isk ? S.k_ts : S.q_ts) +
-                                   (int64_t)hh * (isk ? S.k_hs : S.q_hs);
+        const __nv_bfloat16 *src = (isv ? S.v : isk ? S.k : S.q) +
+                                   t * (isv ? S.v_ts : isk ? S.k_ts : S.q_ts) +
+                                   (int64_t)hh * (isv ? S.v_hs : isk ? S.k_hs : S.q_hs);
         const __nv_bfloat16 *gam = isk ? S.gk : S.gq;
-        __nv_bfloat16 *dst = (isk ? p.k_out : p.q_out) + n * (isk ? p.ko_ts : p.qo_ts) +
-                             (int64_t)hh * D;
+        __nv_bfloat16 *dst = (isv ? p.v_out : isk ? p.k_out : p.q_out) +
+                             n * (isv ? p.vo_ts : isk ? p.ko_ts : p.qo_ts) + (int64_t)hh * D;
 
         float x[NS][8];
+        uint4 raw[NS];
 #pragma unroll
-        for (int k = 0; k < NS; ++k)
-            unpack8((live && vidx[k] >= 0) ? ld_stream(src + 8 * vidx[k]) : make_uint4(0, 0, 0, 0),
-                    x[k]);
+        for (int k = 0; k < NS; ++k) {
+            raw[k] = (live && vidx[k] >= 0) ? ld_stream(src + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
+            unpack8(raw[k], x[k]);
+        }
         if (p.norm) {
             float ss = 0.f;
 #pragma unroll
@@ -129,7 +134,7 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
 #pragma unroll
             for (int k = 0; k < NS; ++k)
                 if (vidx[k] >= 0)
-                    st_stream(dst + 8 * vidx[k], pack8(x[k]));
+                    st_stream(dst + 8 * vidx[k], isv ? raw[k] : pack8(x[k]));
         }
     }
 }

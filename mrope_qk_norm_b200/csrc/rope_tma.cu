@@ -562,6 +562,8 @@ int sm_count()
 cudaError_t launch_rope_tma(const RopeParams &p_in, int layout_paired, int lpr, int ns,
                             int tokens_per_tile, cudaStream_t stream, LaunchRecord *rec)
 {
+    if (p_in.Hv > 0)
+        return cudaErrorNotSupported;  // joint Q/K/V is served by the other kernels
     RopeParams p = p_in;
     const int layout = layout_paired ? PAIRED : VECTOR;
     p.pw = layout == VECTOR ? p.D / 2 : p.P;

@@ -169,6 +169,12 @@ def qk_norm_rope(streams, Hq: int, Hk: int, D: int, rot: int, pairing: int, eps:
     return q_out, k_out
 
 
+def joint_v(v_streams) -> np.ndarray:
+    """V of the joint Q/K/V op (vllm-omni #7600, Purpose): every stream's V
+    rows, unchanged, text first -- the bf16 bit patterns [T0+T1, Hv, D]."""
+    return np.concatenate([bits(v) for v in v_streams], axis=0)
+
+
 def vit_positions(grids, spatial_merge: int) -> np.ndarray:
     """int32 [3, N] (t, h, w) positions of every token, by nested loops."""
     lib = _load()

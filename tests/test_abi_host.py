@@ -157,3 +157,55 @@ def test_fused_refusals(qkr):
     assert call(n=3) == E
     # output stride too small for the heads
     assert call(qots=128) == U
+
+
+def test_fused_qkv_refusals(qkr):
+    E, U = qkr.QKR_ERR_INVALID_ARG, qkr.QKR_ERR_UNSUPPORTED
+    L = qkr.lib()
+    d = qkr.StreamDesc(q=FAKE, k=FAKE + (1 << 20), q_offset=0, k_offset=0, q_tok_stride=256,
+                       q_head_stride=64, k_tok_stride=256, k_head_stride=64, n_tokens=4,
+                       gamma_q=FAKE + (2 << 20), gamma_k=FAKE + (2 << 20), v=FAKE + (7 << 20),
+                       v_offset=0, v_tok_stride=192, v_head_stride=64)
+    a = qkr.AngleDesc(kind=qkr.ANGLE_TABLE, section_mode=0, cos=FAKE + (3 << 20),
+                      sin=FAKE + (4 << 20), table_rows=8, ld=32, plane_stride=256)
+    arr = (qkr.StreamDesc * 2)(d, d)
+
+    def call(n=1, v_out=FAKE + (8 << 20), vots=192, Hv=3):
+        return L.fused_qkv_norm_rope(None, arr, n, FAKE + (5 << 20), FAKE + (6 << 20), v_out,
+                                     256, 256, vots, 4, 4, Hv, 64, 64, 0, 1e-6,
+                                     ctypes.byref(a), 0)
+    # Hv must be >= 1 (the Q/K-only op is fused_qk_norm_rope)
+    assert call(Hv=0) == E and "Hv" in _err(qkr)
+    # v_out missing, misaligned, too narrow, overlapping an input or another output
+    assert call(v_out=0) == E
+    assert call(v_out=FAKE + (8 << 20) + 8) == U
+    assert call(vots=128) == U
+    assert call(v_out=FAKE + (7 << 20)) == U
+    assert call(v_out=FAKE + (5 << 20) + 64) == U
+    # a stream without v
+    arr[0].v = 0
+    assert call() == E and "v must be non-NULL" in _err(qkr)
+    arr[0].v = FAKE + (7 << 20)
+    # v stride not a multiple of 8 elements, v heads overlapping
+    arr[0].v_tok_stride = 196
+    assert call() == U
+    arr[0].v_tok_stride = 192
+    arr[0].v_head_stride = 32
+    assert call() == U
+    arr[0].v_head_stride = 64
+    # an empty call enqueues nothing
+    arr[0].n_tokens = 0
+    assert call() == qkr.QKR_OK
+    assert qkr.last_launch()["launches"] == 0
+
+
+def test_launch_switch_refusals(qkr):
+    L = qkr.lib()
+    assert L.qkr_launch_overlap(2) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_launch_overlap(-1) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(4, 0, 0, 0) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(3, 0, 0, 1) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(3, 5, 0, 0) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(3, 0, 65, 0) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(0, 0, 0, 0) == qkr.QKR_OK
+    assert L.qkr_launch_overlap(1) == qkr.QKR_OK

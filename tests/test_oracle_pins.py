@@ -528,3 +528,18 @@ def test_workload_shapes_match_configs():
     assert [len(w5.inv_t), len(w5.inv_h), len(w5.inv_w)] == [16, 24, 24]
     g = W.config2(R=32, hidden=5120).gamma.float()
     assert float(g.min()) >= 0.5 and float(g.max()) <= 1.5
+
+
+def test_joint_v_is_text_first_row_copy():
+    """V of the joint Q/K/V op: row n of the joint output is row n of the text
+    stream for n < T0, else row n - T0 of the image stream, bit for bit
+    (checked row by row, including an empty text stream)."""
+    g = torch.Generator().manual_seed(5)
+    for T0, T1 in ((3, 5), (0, 4), (6, 0)):
+        a = W.bf16_normal((T0, 2, 8), g)
+        b = W.bf16_normal((T1, 2, 8), g)
+        j = oracle.joint_v([a, b])
+        assert j.shape == (T0 + T1, 2, 8) and j.dtype == np.uint16
+        for n in range(T0 + T1):
+            src = a[n] if n < T0 else b[n - T0]
+            assert np.array_equal(j[n], src.view(torch.int16).numpy().view(np.uint16))
