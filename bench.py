@@ -341,6 +341,24 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
            {"launches_per_step": 2})
     del s4
 
+    # rope + set_rows: config 4's K rows rotated and scattered into a 16384-row cache
+    kb = 8192 * 8 * 128 * 2
+    b_sr = 2 * kb + 8192 * 8 + 3 * 8192 * 4 + 64 * 4
+    g_sr = torch.Generator(device=dev)
+    g_sr.manual_seed(4100)
+    sr_sets = []
+    for _ in range(n_sets_for(b_sr)):
+        x = w4.streams[0].k.to(dev)
+        cache = torch.empty(16384, 8, 128, dtype=torch.bfloat16, device=dev)
+        rid = torch.randperm(16384, generator=g_sr, device=dev)[:8192].contiguous()
+        sr_sets.append((x, cache, rid))
+    record("rope_set_rows", "K 8192 x 8 heads x 128 -> 16384-row cache, interleaved (24,20,20)",
+           [lambda x=x: qkr.rope_set_rows(x[0], x[1], x[2], pos4, inv4, 128,
+                                          W.SECTIONS_INTERLEAVED, (24, 20, 20), 0,
+                                          stream=stream) for x in sr_sets],
+           b_sr, 8192, "tokens")
+    del sr_sets
+
     # config 5: ViT setup and apply, each over rotating output/input sets
     w5 = W.config5()
     g = np.asarray(w5.grids, dtype=np.int64)

@@ -238,6 +238,35 @@ qkr_status mrope_apply(void *stream, const void *q, const void *k, void *q_out, 
                        const void *gamma_q, const void *gamma_k, float eps, uint32_t flags);
 
 /*
+ * rope_set_rows -- rotate K rows and scatter them into cache rows (llama.cpp
+ * fork #286, "The change": the rotation kernels rope_f32 and rope_set_rows_f32
+ * both gain the sectioned mode; the second writes each rotated row into the
+ * destination row its index names, as ggml's ROPE + SET_ROWS pair does when
+ * a decoder stores K in its cache).  For every token t < T and head h:
+ *   cache[row_idx[t], h, :] = rope(norm(x[t, h, :]))
+ * with exactly mrope_apply's angle rules (positions rows, sections, token
+ * offset, pairing) and, when gamma is non-NULL, the per-head RMSNorm first.
+ *
+ *   x                bf16 device [T, H, D], token stride x_tok_stride, heads dense.
+ *   cache            bf16 device [cache_rows, H, D], row stride cache_row_stride
+ *                    (a multiple of 8, >= H*D), heads dense.  Must not overlap x.
+ *   row_idx          int64 device [T], 8-byte aligned: destination row of each
+ *                    token.  Rows must be distinct within a call (two tokens
+ *                    naming one row race).  A row outside [0, cache_rows) is
+ *                    not written and sets bit 4 of the device status word
+ *                    (qkr_device_status); the host cannot see device indices
+ *                    without synchronising, so this is reported, not refused.
+ *   gamma            nullable bf16 [D].
+ * Other arguments, alignment and errors as mrope_apply.
+ */
+qkr_status rope_set_rows(void *stream, const void *x, void *cache, const int64_t *row_idx,
+                         int64_t T, int64_t H, int64_t D, int64_t rot_dim, int64_t x_tok_stride,
+                         int64_t cache_row_stride, int64_t cache_rows, const int32_t *positions,
+                         int64_t n_rows, int64_t T_total, int64_t token_offset,
+                         const float *inv_freq, const int32_t *sections, int32_t section_mode,
+                         int32_t pairing, const void *gamma, float eps, uint32_t flags);
+
+/*
  * vit_mrope_setup -- vLLM mrope_vit_setup (VitMropeSetup.forward and
  * _vit_mrope_setup_kernel): the (3, N, P) fp32 cos/sin t/h/w planes,
  * P = half_t + half_h + half_w.  Token n of grid g (cu_seqlens[g] <= n <
@@ -358,8 +387,9 @@ qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t token
 /* Device status word of the library on the current device (0 = healthy).
  * Kernels that wait on shared-memory barriers give every wait a time budget;
  * a wait that runs out sets a bit here (1: producer, 2: consumer) and the
- * kernel returns early instead of hanging.  Synchronous (copies the word to
- * the host); reset != 0 clears it.  Not for the hot path. */
+ * kernel returns early instead of hanging.  Bit 4: rope_set_rows met a row
+ * index outside the cache (that row was not written).  Synchronous (copies
+ * the word to the host); reset != 0 clears it.  Not for the hot path. */
 qkr_status qkr_device_status(uint32_t *status, int32_t reset);
 
 /* Writes the axis (0 t, 1 h, 2 w, 3 e) of pairs 0..P-1 under a section mode

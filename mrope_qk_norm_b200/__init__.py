@@ -27,7 +27,7 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
                 4: "vit_setup", 5: "rms_rows", 6: "rms_cluster", 7: "section_map",
                 8: "vit_positions"}
 
-EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "vit_mrope_setup", "rms_norm_residual",
+EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "rope_set_rows", "vit_mrope_setup", "rms_norm_residual",
            "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
            "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status", "qkr_launch_overlap")
 
@@ -83,6 +83,8 @@ def _load() -> ctypes.CDLL:
                                 I64, I64, I64, I64, I32, F, ctypes.POINTER(AngleDesc), U32],
         "mrope_apply": [V, V, V, V, V, I64, I64, I64, I64, I64, I64, I64, I64, I64, V, I64, I64,
                         I64, V, V, I32, I32, V, V, F, U32],
+        "rope_set_rows": [V, V, V, V, I64, I64, I64, I64, I64, I64, I64, V, I64, I64, I64, V, V,
+                          I32, I32, V, F, U32],
         "vit_mrope_setup": [V, V, V, V, I64, I64, I64, V, V, I64, I64, I64, V, V],
         "rms_norm_residual": [V, V, V, V, V, I64, I64, I64, I64, I64, F],
         "qkr_last_launch": [ctypes.POINTER(LaunchInfo)],
@@ -319,6 +321,36 @@ def mrope_apply(q, k, q_out, k_out, positions, inv_freq, rot_dim, section_mode=S
         eps, flags))
 
 
+
+
+def rope_set_rows(x, cache, row_idx, positions, inv_freq, rot_dim, section_mode=SECTIONS_NONE,
+                  sections=None, pairing=PAIRING_NEOX, token_offset=0, gamma=None, eps=1e-6,
+                  flags=0, stream=None):
+    """cache[row_idx[t]] = rope(norm(x[t])): x [T, H, D] bf16 (heads dense),
+    cache [R, H, D] bf16 (heads dense), row_idx int64 [T]; positions int32
+    [rows, T_total]."""
+    for name, t in (("x", x), ("cache", cache)):
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("%s must be [T, H, D] with dense heads" % name)
+    if x.shape[1:] != cache.shape[1:]:
+        raise ValueError("x and cache must have the same heads and head dim")
+    if row_idx.dim() != 1 or row_idx.shape[0] != x.shape[0] or row_idx.stride(0) != 1:
+        raise ValueError("row_idx must be a contiguous int64 [T] tensor")
+    if positions.dim() == 1:
+        positions = positions.view(1, -1)
+    if not positions.is_contiguous():
+        raise ValueError("positions must be contiguous [rows, T_total]")
+    sec = None
+    if sections is not None:
+        sec = (ctypes.c_int32 * 4)(*(list(sections) + [0] * (4 - len(sections))))
+    T, H, D = x.shape
+    _check(_lib.rope_set_rows(
+        _stream(stream), _ptr(x, torch.bfloat16, "x"), _ptr(cache, torch.bfloat16, "cache"),
+        _ptr(row_idx, torch.int64, "row_idx"), T, H, D, rot_dim, x.stride(0), cache.stride(0),
+        cache.shape[0], _ptr(positions, torch.int32, "positions"), positions.shape[0],
+        positions.shape[1], token_offset, _ptr(inv_freq, torch.float32, "inv_freq"),
+        ctypes.cast(sec, ctypes.c_void_p) if sec is not None else None, section_mode, pairing,
+        _ptr(gamma, torch.bfloat16, "gamma") if gamma is not None else None, eps, flags))
 # --------------------------------------------------------------------------
 # vit_mrope_setup
 # --------------------------------------------------------------------------

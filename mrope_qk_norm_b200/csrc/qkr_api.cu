@@ -170,9 +170,9 @@ qkr_status check_angle(const qkr_angle_desc *a, int64_t P, int64_t T, qkr::RopeP
 }
 
 qkr_status check_geometry(int64_t Hq, int64_t Hk, int64_t D, int64_t rot, int32_t pairing,
-                          float eps)
+                          float eps, bool k_only = false)
 {
-    if (Hq < 1 || Hk < 1 || Hq + Hk > 65536)
+    if (Hq < (k_only ? 0 : 1) || Hk < 1 || Hq + Hk > 65536)
         return fail(QKR_ERR_INVALID_ARG, "head counts must be >= 1 and Hq + Hk <= 65536");
     if (D < 8 || D > 256 || D % 8)
         return fail(QKR_ERR_UNSUPPORTED, "head_dim %lld: need a multiple of 8 in [8, 256]",
@@ -194,11 +194,19 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
                      void *q_out, void *k_out, int64_t qo_ts, int64_t ko_ts, int64_t Hq,
                      int64_t Hk, int64_t D, int64_t rot, int32_t pairing, float eps,
                      const qkr_angle_desc *angle, uint32_t flags, bool norm, bool inplace_ok,
-                     int64_t Hv = 0, void *v_out = nullptr, int64_t vo_ts = 0)
+                     int64_t Hv = 0, void *v_out = nullptr, int64_t vo_ts = 0,
+                     bool k_only = false, const int64_t *k_rows = nullptr,
+                     int64_t k_out_rows = 0)
 {
-    qkr_status st = check_geometry(Hq, Hk, D, rot, pairing, eps);
+    // k_only: K-only scatter (rope_set_rows): no Q heads, K row n goes to
+    // output row k_rows[n] of a k_out buffer with k_out_rows rows.
+    qkr_status st = check_geometry(Hq, Hk, D, rot, pairing, eps, k_only);
     if (st != QKR_OK)
         return st;
+    if (k_only && (Hq != 0 || Hv != 0 || k_out_rows < 1 || k_out_rows > ((int64_t)1 << 40)))
+        return fail(QKR_ERR_INVALID_ARG, "scatter: need Hq == 0, no V and 1 <= cache rows");
+    if (k_only && (reinterpret_cast<uintptr_t>(k_rows) & 7u))
+        return fail(QKR_ERR_UNSUPPORTED, "row indices must be 8-byte aligned");
     if (Hv < 0 || Hq + Hk + Hv > 65536)
         return fail(QKR_ERR_INVALID_ARG, "V head count out of range");
     if (!streams || n_streams < 1 || n_streams > 2)
@@ -216,11 +224,11 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
         g_error.clear();
         return QKR_OK;
     }
-    if (!q_out || !k_out)
+    if ((Hq > 0 && !q_out) || !k_out)
         return fail(QKR_ERR_INVALID_ARG, "q_out and k_out must be non-NULL");
-    if (!aligned16(q_out) || !aligned16(k_out))
+    if ((Hq > 0 && !aligned16(q_out)) || !aligned16(k_out))
         return fail(QKR_ERR_UNSUPPORTED, "outputs must be 16-byte aligned");
-    if (qo_ts < Hq * D || ko_ts < Hk * D || qo_ts % 8 || ko_ts % 8)
+    if ((Hq > 0 && (qo_ts < Hq * D || qo_ts % 8)) || ko_ts < Hk * D || ko_ts % 8)
         return fail(QKR_ERR_UNSUPPORTED,
                     "output token strides must be multiples of 8 and hold a token's heads");
     if (Hv > 0) {
@@ -246,38 +254,45 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
             p.st[s] = qkr::RopeStreamDev{};
             continue;
         }
-        if (!d.q || !d.k)
+        qkr_stream_desc dd = d;
+        if (Hq == 0) {  // K-only call: Q is never read
+            dd.q = d.k;
+            dd.q_offset = d.k_offset;
+            dd.q_tok_stride = d.k_tok_stride;
+            dd.q_head_stride = d.k_head_stride;
+        }
+        if (!dd.q || !d.k)
             return fail(QKR_ERR_INVALID_ARG, "stream %d: q and k must be non-NULL", s);
-        if (d.q_offset < 0 || d.k_offset < 0)
+        if (dd.q_offset < 0 || d.k_offset < 0)
             return fail(QKR_ERR_INVALID_ARG, "stream %d: storage offsets must be >= 0", s);
-        if (d.q_tok_stride <= 0 || d.k_tok_stride <= 0 || d.q_head_stride < D ||
+        if (dd.q_tok_stride <= 0 || d.k_tok_stride <= 0 || dd.q_head_stride < D ||
             d.k_head_stride < D)
             return fail(QKR_ERR_UNSUPPORTED,
                         "stream %d: strides must be positive and heads must not overlap", s);
-        if (d.q_tok_stride % 8 || d.k_tok_stride % 8 || d.q_head_stride % 8 ||
-            d.k_head_stride % 8 || d.q_offset % 8 || d.k_offset % 8)
+        if (dd.q_tok_stride % 8 || d.k_tok_stride % 8 || dd.q_head_stride % 8 ||
+            d.k_head_stride % 8 || dd.q_offset % 8 || d.k_offset % 8)
             return fail(QKR_ERR_UNSUPPORTED,
                         "stream %d: offsets and strides must be multiples of 8 elements "
                         "(16-byte vectors)", s);
-        if (!view_fits(d.n_tokens, d.q_tok_stride, Hq, d.q_head_stride, D) ||
+        if (!view_fits(d.n_tokens, dd.q_tok_stride, Hq, dd.q_head_stride, D) ||
             !view_fits(d.n_tokens, d.k_tok_stride, Hk, d.k_head_stride, D) ||
-            d.q_offset > ((int64_t)1 << 60) || d.k_offset > ((int64_t)1 << 60))
+            dd.q_offset > ((int64_t)1 << 60) || d.k_offset > ((int64_t)1 << 60))
             return fail(QKR_ERR_INVALID_ARG, "stream %d: view exceeds the address range", s);
-        qb[s] = static_cast<const __nv_bfloat16 *>(d.q) + d.q_offset;
+        qb[s] = static_cast<const __nv_bfloat16 *>(dd.q) + dd.q_offset;
         kb[s] = static_cast<const __nv_bfloat16 *>(d.k) + d.k_offset;
         if (!aligned16(qb[s]) || !aligned16(kb[s]))
             return fail(QKR_ERR_UNSUPPORTED, "stream %d: q/k must be 16-byte aligned", s);
         if (norm) {
-            if (!d.gamma_q || !d.gamma_k)
+            if ((Hq > 0 && !d.gamma_q) || !d.gamma_k)
                 return fail(QKR_ERR_INVALID_ARG, "stream %d: gamma_q and gamma_k are required",
                             s);
-            if (!aligned16(d.gamma_q) || !aligned16(d.gamma_k))
+            if ((Hq > 0 && !aligned16(d.gamma_q)) || !aligned16(d.gamma_k))
                 return fail(QKR_ERR_UNSUPPORTED, "stream %d: gammas must be 16-byte aligned", s);
         }
         p.st[s].q = qb[s];
         p.st[s].k = kb[s];
-        p.st[s].q_ts = d.q_tok_stride;
-        p.st[s].q_hs = d.q_head_stride;
+        p.st[s].q_ts = dd.q_tok_stride;
+        p.st[s].q_hs = dd.q_head_stride;
         p.st[s].k_ts = d.k_tok_stride;
         p.st[s].k_hs = d.k_head_stride;
         p.st[s].gq = static_cast<const __nv_bfloat16 *>(d.gamma_q);
@@ -308,12 +323,13 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     }
     if (T > ((int64_t)1 << 40))
         return fail(QKR_ERR_INVALID_ARG, "token count too large");
-    if (!view_fits(T, qo_ts, 1, 0, Hq * D) || !view_fits(T, ko_ts, 1, 0, Hk * D))
+    const int64_t k_rows_out = k_only ? k_out_rows : T;
+    if (!view_fits(T, qo_ts, 1, 0, Hq * D) || !view_fits(k_rows_out, ko_ts, 1, 0, Hk * D))
         return fail(QKR_ERR_INVALID_ARG, "output view exceeds the address range");
 
     // Aliasing: outputs may equal inputs only where allowed, never overlap otherwise.
     const Span so_q = view_span(q_out, T, qo_ts, Hq, D, D);
-    const Span so_k = view_span(k_out, T, ko_ts, Hk, D, D);
+    const Span so_k = view_span(k_out, k_rows_out, ko_ts, Hk, D, D);
     if (overlap(so_q, so_k))
         return fail(QKR_ERR_UNSUPPORTED, "q_out and k_out overlap");
     Span so_v;
@@ -371,6 +387,13 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     p.rot = (int)rot;
     p.P = (int)P;
     p.rows_per_token = (int)(Hq + Hk + Hv);
+    p.k_rows = k_rows;
+    p.k_out_rows = k_only ? k_out_rows : 0;
+    if (k_only) {
+        cudaError_t se = qkr::device_status_address(&p.status);
+        if (se != cudaSuccess)
+            return cuda_result(se, "device status address");
+    }
     p.eps = eps;
     p.inv_D = 1.0f / (float)D;
     p.norm = norm ? 1 : 0;
@@ -537,6 +560,48 @@ static qkr_status vit_common(const int32_t *cu, const int32_t *grids, int64_t G,
     p.N = N;
     p.m = (int)m;
     return QKR_OK;
+}
+
+qkr_status rope_set_rows(void *stream, const void *x, void *cache, const int64_t *row_idx,
+                         int64_t T, int64_t H, int64_t D, int64_t rot_dim, int64_t x_tok_stride,
+                         int64_t cache_row_stride, int64_t cache_rows, const int32_t *positions,
+                         int64_t n_rows, int64_t T_total, int64_t token_offset,
+                         const float *inv_freq, const int32_t *sections, int32_t section_mode,
+                         int32_t pairing, const void *gamma, float eps, uint32_t flags)
+{
+    const bool norm = gamma != nullptr;
+    if (!norm && (flags & QKR_FLAG_ROUND_NORMALIZED_BF16))
+        return fail(QKR_ERR_INVALID_ARG, "ROUND_NORMALIZED_BF16 needs normalisation (gamma)");
+    if (section_mode < QKR_SECTIONS_NONE || section_mode > QKR_SECTIONS_IMROPE)
+        return fail(QKR_ERR_INVALID_ARG, "unknown section mode %d", section_mode);
+    if (rot_dim > 0 && n_rows != rows_for_mode(section_mode))
+        return fail(QKR_ERR_INVALID_ARG, "section mode %d reads %d position rows, got %lld",
+                    section_mode, rows_for_mode(section_mode), (long long)n_rows);
+    if (section_mode != QKR_SECTIONS_NONE && !sections)
+        return fail(QKR_ERR_INVALID_ARG,
+                    "section mode %d needs its sections: refusing rather than rotating every "
+                    "pair by one row", section_mode);
+    if (T > 0 && !row_idx)
+        return fail(QKR_ERR_INVALID_ARG, "row_idx must be non-NULL");
+    qkr_stream_desc d = {};
+    d.k = x;
+    d.k_tok_stride = x_tok_stride;
+    d.k_head_stride = D;
+    d.n_tokens = T;
+    d.gamma_k = gamma;
+    qkr_angle_desc a = {};
+    a.kind = QKR_ANGLE_POSITIONS;
+    a.section_mode = section_mode;
+    if (sections)
+        for (int i = 0; i < 4; ++i)
+            a.sections[i] = sections[i];
+    a.positions = positions;
+    a.pos_row_stride = T_total;
+    a.inv_freq = inv_freq;
+    a.token_offset = token_offset;
+    return rope_call(stream, &d, 1, nullptr, cache, 0, cache_row_stride, 0, H, D, rot_dim,
+                     pairing, eps, &a, flags, norm, /*inplace_ok=*/false, 0, nullptr, 0,
+                     /*k_only=*/true, row_idx, cache_rows);
 }
 
 qkr_status vit_mrope_setup(void *stream, const float *inv_t, const float *inv_h,

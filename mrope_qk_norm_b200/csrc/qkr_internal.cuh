@@ -175,6 +175,9 @@ struct RopeParams {
     const float *sin;
     int64_t ld, plane_stride;
     int tab_vec4;             // table bases 16-byte aligned, ld and plane_stride % 4 == 0
+    const int64_t *k_rows;    // scatter: output row of each K token (NULL: row n)
+    int64_t k_out_rows;       // scatter: rows of k_out
+    unsigned *status;         // device status word (scatter: out-of-range rows)
     int stages;               // streaming kernel: depth of the cp.async row ring
     int64_t token_offset;
 };
@@ -198,6 +201,8 @@ cudaError_t launch_rope_tma(const RopeParams &p, int layout_paired, int lpr, int
 // Reads (and optionally clears) the device status word that bounded waits set
 // on timeout.  Synchronous.
 cudaError_t read_device_status(unsigned *status, bool reset);
+// Device address of that status word on the current device.
+cudaError_t device_status_address(unsigned **addr);
 
 // Each launcher enqueues exactly one kernel and returns the CUDA launch status.
 cudaError_t launch_rope_rows(const RopeParams &p, int pairing, cudaStream_t stream,

@@ -161,7 +161,19 @@ __device__ __forceinline__ Item decode_item(const RopeParams &p, int64_t tok0, i
     const int64_t ts = r.isk ? S.k_ts : S.q_ts;
     r.hs = r.isk ? S.k_hs : S.q_hs;
     r.src = base + t * ts + (int64_t)h0 * r.hs;
-    r.dst = (r.isk ? p.k_out : p.q_out) + n * (r.isk ? p.ko_ts : p.qo_ts) + (int64_t)h0 * p.D;
+    // K scatter (rope_set_rows): row n of K goes to output row k_rows[n]; a row
+    // outside the output is not written and raises bit 4 of the status word
+    int64_t orow = n;
+    if (r.isk && p.k_rows && live) {
+        orow = __ldg(reinterpret_cast<const long long *>(p.k_rows) + n);
+        if (orow < 0 || orow >= p.k_out_rows) {
+            atomicOr(p.status, 4u);
+            r.nh = 0;
+            orow = 0;
+        }
+    }
+    r.dst = (r.isk ? p.k_out : p.q_out) + orow * (r.isk ? p.ko_ts : p.qo_ts) +
+            (int64_t)h0 * p.D;
     return r;
 }
 

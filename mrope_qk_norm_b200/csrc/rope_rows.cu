@@ -69,8 +69,18 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
                                    t * (isv ? S.v_ts : isk ? S.k_ts : S.q_ts) +
                                    (int64_t)hh * (isv ? S.v_hs : isk ? S.k_hs : S.q_hs);
         const __nv_bfloat16 *gam = isk ? S.gk : S.gq;
+        int64_t orow = n;
+        bool write = live;
+        if (isk && p.k_rows && live) {  // K scatter (rope_set_rows)
+            orow = __ldg(reinterpret_cast<const long long *>(p.k_rows) + n);
+            if (orow < 0 || orow >= p.k_out_rows) {
+                atomicOr(p.status, 4u);
+                write = false;
+                orow = 0;
+            }
+        }
         __nv_bfloat16 *dst = (isv ? p.v_out : isk ? p.k_out : p.q_out) +
-                             n * (isv ? p.vo_ts : isk ? p.ko_ts : p.qo_ts) + (int64_t)hh * D;
+                             orow * (isv ? p.vo_ts : isk ? p.ko_ts : p.qo_ts) + (int64_t)hh * D;
 
         float x[NS][8];
         uint4 raw[NS];
@@ -130,7 +140,7 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
             }
         }
         __syncwarp();
-        if (live) {
+        if (write) {
 #pragma unroll
             for (int k = 0; k < NS; ++k)
                 if (vidx[k] >= 0)

@@ -562,6 +562,8 @@ int sm_count()
 cudaError_t launch_rope_tma(const RopeParams &p_in, int layout_paired, int lpr, int ns,
                             int tokens_per_tile, cudaStream_t stream, LaunchRecord *rec)
 {
+    if (p_in.k_rows)
+        return cudaErrorNotSupported;  // the scatter is served by the other kernels
     if (p_in.Hv > 0)
         return cudaErrorNotSupported;  // joint Q/K/V is served by the other kernels
     RopeParams p = p_in;
@@ -651,6 +653,14 @@ cudaError_t launch_rope_tma(const RopeParams &p_in, int layout_paired, int lpr, 
         rec->launches = 1;
         rec->pipelined = 1;
     }
+    return e;
+}
+
+cudaError_t device_status_address(unsigned **addr)
+{
+    void *a = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&a, g_device_error);
+    *addr = static_cast<unsigned *>(a);
     return e;
 }
 

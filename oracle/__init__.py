@@ -175,6 +175,17 @@ def joint_v(v_streams) -> np.ndarray:
     return np.concatenate([bits(v) for v in v_streams], axis=0)
 
 
+def scatter_rows(rows: np.ndarray, row_idx, n_rows: int, fill=np.nan) -> np.ndarray:
+    """rope_set_rows's destination (llama.cpp fork #286, "The change": rotated
+    rows written to the rows their indices name): out[row_idx[t]] = rows[t];
+    rows no index names hold `fill`."""
+    idx = np.asarray(row_idx, dtype=np.int64)
+    out = np.full((n_rows,) + rows.shape[1:], fill, dtype=rows.dtype)
+    for t, r in enumerate(idx):
+        out[r] = rows[t]
+    return out
+
+
 def vit_positions(grids, spatial_merge: int) -> np.ndarray:
     """int32 [3, N] (t, h, w) positions of every token, by nested loops."""
     lib = _load()

@@ -209,3 +209,24 @@ def test_launch_switch_refusals(qkr):
     assert L.qkr_tune_rope(3, 0, 65, 0) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(0, 0, 0, 0) == qkr.QKR_OK
     assert L.qkr_launch_overlap(1) == qkr.QKR_OK
+
+
+def test_rope_set_rows_refusals(qkr):
+    E, U = qkr.QKR_ERR_INVALID_ARG, qkr.QKR_ERR_UNSUPPORTED
+    L = qkr.lib()
+    sec = ctypes.cast((ctypes.c_int32 * 4)(24, 20, 20, 0), ctypes.c_void_p)
+
+    def call(x=FAKE, cache=FAKE + (1 << 20), rows=FAKE + (2 << 20), T=4, R=16, cstride=1024,
+             n_rows=3, mode=qkr.SECTIONS_INTERLEAVED, gamma=None, flags=0):
+        return L.rope_set_rows(None, x, cache, rows, T, 8, 128, 128, 1024, cstride, R,
+                               FAKE + (3 << 20), n_rows, 4, 0, FAKE + (4 << 20), sec, mode, 0,
+                               gamma, 1e-6, flags)
+    assert call(rows=None) == E and "row_idx" in _err(qkr)
+    assert call(rows=FAKE + (2 << 20) + 4) == U        # not 8-byte aligned
+    assert call(R=0) == E                               # empty cache
+    assert call(cache=FAKE + 512) == U                  # cache overlaps x
+    assert call(cstride=1000) == U                      # row stride not a multiple of 8
+    assert call(n_rows=1) == E                          # interleaved mode reads 3 rows
+    assert call(flags=qkr.FLAG_ROUND_NORMALIZED_BF16) == E  # rounding contract needs gamma
+    assert call(T=0, rows=None) == qkr.QKR_OK           # empty: nothing enqueued
+    assert qkr.last_launch()["launches"] == 0

@@ -543,3 +543,17 @@ def test_joint_v_is_text_first_row_copy():
         for n in range(T0 + T1):
             src = a[n] if n < T0 else b[n - T0]
             assert np.array_equal(j[n], src.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_scatter_rows_places_each_row_once():
+    """rope_set_rows's destination: brute-force row placement on a tiny case,
+    including unnamed rows (fill) and a reversed index order."""
+    rows = np.arange(4 * 2 * 3, dtype=np.float64).reshape(4, 2, 3)
+    idx = [6, 0, 3, 1]
+    out = oracle.scatter_rows(rows, idx, 8, fill=-1.0)
+    for t, r in enumerate(idx):
+        assert np.array_equal(out[r], rows[t])
+    for r in set(range(8)) - set(idx):
+        assert (out[r] == -1.0).all()
+    rev = oracle.scatter_rows(rows, [3, 2, 1, 0], 4)
+    assert np.array_equal(rev, rows[::-1])
