@@ -408,6 +408,15 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
         record("rms_norm_residual", "R=%d hidden=%d" % (R, hidden),
                [lambda s=s: qkr.rms_norm_residual(s[0], s[1], s[2], s[3], 1e-6, stream)
                 for s in sets], nb, R, "rows")
+        if R in (1, 1024, 16384) and hidden == 8192 or R == 1:
+            # the static-FP8 output variant: out is one byte per element
+            nb8 = 7 * R * hidden + 2 * hidden + 4
+            sc = torch.tensor([0.05], dtype=torch.float32, device=dev)
+            outs8 = [torch.empty(R, hidden, dtype=torch.uint8, device=dev) for _ in sets]
+            record("rms_norm_fp8", "R=%d hidden=%d, FP8 E4M3 out" % (R, hidden),
+                   [lambda s=s, o=o: qkr.rms_norm_fp8(s[0], s[1], s[2], o, sc, 1e-6, stream)
+                    for s, o in zip(sets, outs8)], nb8, R, "rows")
+            del outs8
         del sets
     torch.cuda.synchronize()
     return rows

@@ -1,7 +1,8 @@
 /*
  * qkr.h -- C ABI of the B200 (sm_100a) normalise-then-rotate library.
  *
- * Four operations, each one CUDA kernel launch on the caller's stream:
+ * The four operations of the path and their extensions, each one CUDA kernel
+ * launch on the caller's stream:
  *
  *   fused_qk_norm_rope  per-head RMSNorm of Q and K, optional text/image
  *                       concatenation, RoPE (NeoX or GPT-J pairing), one launch.
@@ -14,6 +15,9 @@
  *                       per-image [t, h, w] grids.
  *   rms_norm_residual   hidden-size RMSNorm with a fused residual add; splits
  *                       one row across a thread-block cluster when rows are few.
+ *   rms_norm_fp8        the same with a static-scale FP8 E4M3 output.
+ *   rope_set_rows       mrope_apply's rotation of K rows, scattered into cache
+ *                       rows by index.
  *
  * Conventions shared by every entry point:
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
@@ -312,6 +316,26 @@ qkr_status vit_mrope_setup(void *stream, const float *inv_t, const float *inv_h,
 qkr_status rms_norm_residual(void *stream, const void *x, void *residual, const void *gamma,
                              void *out, int64_t R, int64_t hidden, int64_t x_stride,
                              int64_t res_stride, int64_t out_stride, float eps);
+
+/*
+ * rms_norm_fp8 -- rms_norm_residual with a static FP8 output (vLLM #26234,
+ * Purpose: the same vectorised variance read serves rms_norm_kernel and
+ * rms_norm_static_fp8_quant_kernel).  With a residual, s = bf16(x + residual)
+ * is written back to residual as in rms_norm_residual; without one
+ * (residual == NULL) s = x.  Then y = s * rsqrt(mean(s^2) + eps) * gamma in
+ * fp32, and out holds the FP8 E4M3 (OCP "FN": no infinities, max 448) code of
+ * y / scale, rounded to nearest even and saturated to +-448.
+ *
+ *   out              device uint8 [R, hidden] E4M3 codes, row stride out_stride
+ *                    bytes (a multiple of 8), 8-byte aligned.
+ *   scale            device fp32 [1]: the static per-tensor scale (read on the
+ *                    device, so the call never synchronises).
+ *   residual         nullable; res_stride is ignored when NULL.
+ * Other arguments and errors as rms_norm_residual; out must not overlap any input.
+ */
+qkr_status rms_norm_fp8(void *stream, const void *x, void *residual, const void *gamma,
+                        void *out, const float *scale, int64_t R, int64_t hidden,
+                        int64_t x_stride, int64_t res_stride, int64_t out_stride, float eps);
 
 /* ------------------------------------------------------------------------
  * Introspection and debug entry points (used by the tests).

@@ -27,8 +27,8 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
                 4: "vit_setup", 5: "rms_rows", 6: "rms_cluster", 7: "section_map",
                 8: "vit_positions"}
 
-EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "rope_set_rows", "vit_mrope_setup", "rms_norm_residual",
-           "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
+EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "rope_set_rows",
+           "vit_mrope_setup", "rms_norm_residual", "rms_norm_fp8", "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
            "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status", "qkr_launch_overlap")
 
 
@@ -87,6 +87,7 @@ def _load() -> ctypes.CDLL:
                           I32, I32, V, F, U32],
         "vit_mrope_setup": [V, V, V, V, I64, I64, I64, V, V, I64, I64, I64, V, V],
         "rms_norm_residual": [V, V, V, V, V, I64, I64, I64, I64, I64, F],
+        "rms_norm_fp8": [V, V, V, V, V, V, I64, I64, I64, I64, I64, F],
         "qkr_last_launch": [ctypes.POINTER(LaunchInfo)],
         "qkr_section_map": [V, I32, V, I64, V],
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
@@ -400,3 +401,22 @@ def vit_positions(cu_seqlens, grids, n_tokens, spatial_merge, out, stream=None):
     _check(_lib.qkr_vit_positions(_stream(stream), _ptr(cu_seqlens, torch.int32, "cu_seqlens"),
                                   _ptr(grids, torch.int32, "grids"), grids.shape[0], n_tokens,
                                   spatial_merge, _ptr(out, torch.int32, "pos_out")))
+
+
+def rms_norm_fp8(x, residual, gamma, out, scale, eps, stream=None):
+    """x: [R, hidden] bf16; residual: [R, hidden] bf16 updated in place, or None;
+    out: [R, hidden] uint8 (E4M3 codes; view as torch.float8_e4m3fn); scale:
+    fp32 [1] device tensor."""
+    for name, t in (("x", x), ("out", out)) + ((("residual", residual),) if residual is not None else ()):
+        if t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError("%s must be [R, hidden] with a contiguous hidden dim" % name)
+    if out.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("out must be uint8 or float8_e4m3fn")
+    if scale.dtype != torch.float32 or scale.numel() != 1 or not scale.is_cuda:
+        raise ValueError("scale must be a one-element fp32 CUDA tensor")
+    R, hidden = x.shape
+    _check(_lib.rms_norm_fp8(
+        _stream(stream), _ptr(x, torch.bfloat16, "x"),
+        _ptr(residual, torch.bfloat16, "residual") if residual is not None else None,
+        _ptr(gamma, torch.bfloat16, "gamma"), out.data_ptr(), scale.data_ptr(), R, hidden,
+        x.stride(0), residual.stride(0) if residual is not None else 0, out.stride(0), eps))

@@ -681,7 +681,7 @@ qkr_status rms_norm_residual(void *stream, const void *x, void *residual, const 
         return fail(QKR_ERR_UNSUPPORTED, "residual must not overlap x or out");
     if (overlap(sx, so) && !(x == out && x_stride == out_stride))
         return fail(QKR_ERR_UNSUPPORTED, "out may only alias x exactly (same stride)");
-    qkr::RmsParams p;
+    qkr::RmsParams p = {};
     p.x = static_cast<const __nv_bfloat16 *>(x);
     p.res = static_cast<__nv_bfloat16 *>(residual);
     p.gamma = static_cast<const __nv_bfloat16 *>(gamma);
@@ -697,6 +697,71 @@ qkr_status rms_norm_residual(void *stream, const void *x, void *residual, const 
     qkr_status r = cuda_result(
         qkr::launch_rms_norm_residual(p, static_cast<cudaStream_t>(stream), &rec),
         "rms norm launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
+}
+
+qkr_status rms_norm_fp8(void *stream, const void *x, void *residual, const void *gamma,
+                        void *out, const float *scale, int64_t R, int64_t hidden,
+                        int64_t x_stride, int64_t res_stride, int64_t out_stride, float eps)
+{
+    if (R < 0)
+        return fail(QKR_ERR_INVALID_ARG, "R must be >= 0");
+    if (hidden < 8 || hidden > 65536 || hidden % 8)
+        return fail(QKR_ERR_UNSUPPORTED, "hidden %lld: need a multiple of 8 in [8, 65536]",
+                    (long long)hidden);
+    if (!(eps >= 0.f) || eps > 1.f)
+        return fail(QKR_ERR_INVALID_ARG, "eps must be finite and in [0, 1]");
+    if (R == 0) {
+        g_last = qkr::LaunchRecord();
+        g_error.clear();
+        return QKR_OK;
+    }
+    if (R > ((int64_t)1 << 31) - 1)
+        return fail(QKR_ERR_INVALID_ARG, "too many rows");
+    if (!x || !gamma || !out || !scale)
+        return fail(QKR_ERR_INVALID_ARG, "x, gamma, out and scale must be non-NULL");
+    if (!aligned16(x) || (residual && !aligned16(residual)) || !aligned16(gamma) ||
+        (reinterpret_cast<uintptr_t>(out) & 7u) || !aligned4(scale))
+        return fail(QKR_ERR_UNSUPPORTED,
+                    "x, residual, gamma 16-byte aligned; out 8-byte; scale 4-byte");
+    if (x_stride < hidden || x_stride % 8 || out_stride < hidden || out_stride % 8 ||
+        (residual && (res_stride < hidden || res_stride % 8)))
+        return fail(QKR_ERR_UNSUPPORTED,
+                    "row strides must be >= hidden and multiples of 8 elements");
+    if (!view_fits(R, x_stride, 1, 0, hidden) || !view_fits(R, out_stride, 1, 0, hidden) ||
+        (residual && !view_fits(R, res_stride, 1, 0, hidden)))
+        return fail(QKR_ERR_INVALID_ARG, "view exceeds the address range");
+    const Span sx = view_span(x, R, x_stride, 1, 0, hidden);
+    Span so;  // FP8 rows: one byte per element
+    so.lo = reinterpret_cast<uintptr_t>(out);
+    so.hi = so.lo + (uintptr_t)((R - 1) * out_stride + hidden);
+    const Span ss{reinterpret_cast<uintptr_t>(scale), reinterpret_cast<uintptr_t>(scale) + 4};
+    if (overlap(sx, so) || overlap(so, ss))
+        return fail(QKR_ERR_UNSUPPORTED, "out must not overlap x or scale");
+    if (residual) {
+        const Span sr = view_span(residual, R, res_stride, 1, 0, hidden);
+        if (overlap(sr, so) || overlap(sr, sx) || overlap(sr, ss))
+            return fail(QKR_ERR_UNSUPPORTED, "residual must not overlap x, out or scale");
+    }
+    qkr::RmsParams p = {};
+    p.x = static_cast<const __nv_bfloat16 *>(x);
+    p.res = static_cast<__nv_bfloat16 *>(residual);
+    p.gamma = static_cast<const __nv_bfloat16 *>(gamma);
+    p.out8 = static_cast<uint8_t *>(out);
+    p.scale = scale;
+    p.R = R;
+    p.hidden = (int)hidden;
+    p.xs = x_stride;
+    p.rs = res_stride;
+    p.os = out_stride;
+    p.eps = eps;
+    p.inv_hidden = 1.0f / (float)hidden;
+    qkr::LaunchRecord rec;
+    qkr_status r = cuda_result(
+        qkr::launch_rms_norm_residual(p, static_cast<cudaStream_t>(stream), &rec),
+        "rms norm fp8 launch");
     if (r == QKR_OK)
         g_last = rec;
     return r;

@@ -228,9 +228,11 @@ cudaError_t launch_section_map(int mode, const int (&sec)[4], int P, int8_t *out
 
 struct RmsParams {
     const __nv_bfloat16 *x;
-    __nv_bfloat16 *res;
+    __nv_bfloat16 *res;       // NULL (FP8 variant only): no residual add
     const __nv_bfloat16 *gamma;
-    __nv_bfloat16 *out;
+    __nv_bfloat16 *out;       // bf16 output (rms_norm_residual)
+    uint8_t *out8;            // FP8 E4M3 output (rms_norm_fp8)
+    const float *scale;       // FP8: static per-tensor scale (device fp32 [1])
     int64_t R;
     int hidden;
     int64_t xs, rs, os;

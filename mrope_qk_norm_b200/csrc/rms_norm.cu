@@ -17,6 +17,7 @@
 // on a flag: the cluster barrier's co-residency is guaranteed by the hardware.
 
 #include <cooperative_groups.h>
+#include <cuda_fp8.h>
 
 #include <climits>
 
@@ -48,24 +49,21 @@ __device__ __forceinline__ float block_sum(float v, float *red)
 
 // Loads the slice [v0, v1) of a row (vector units), forms s = bf16(x + res),
 // writes it back to residual and returns the fp32 sum of s^2 of this thread.
+// Without a residual (p.res == NULL, FP8 variant) s = x.
 template <int VPT>
 __device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v0, int v1,
                                           float (&s)[VPT][8], bool (&live)[VPT])
 {
     const __nv_bfloat16 *xr = p.x + row * p.xs;
-    __nv_bfloat16 *rr = p.res + row * p.rs;
+    const bool has_res = p.res != nullptr;
+    __nv_bfloat16 *rr = has_res ? p.res + row * p.rs : nullptr;
     uint4 xv[VPT], rv[VPT];
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         const int v = v0 + threadIdx.x + k * blockDim.x;
         live[k] = v < v1;
-        if (live[k]) {
-            xv[k] = ld_stream(xr + 8 * v);
-            rv[k] = ld_stream(rr + 8 * v);
-        } else {
-            xv[k] = make_uint4(0, 0, 0, 0);
-            rv[k] = xv[k];
-        }
+        xv[k] = live[k] ? ld_stream(xr + 8 * v) : make_uint4(0, 0, 0, 0);
+        rv[k] = live[k] && has_res ? ld_stream(rr + 8 * v) : make_uint4(0, 0, 0, 0);
     }
     float ss = 0.f;
 #pragma unroll
@@ -81,18 +79,22 @@ __device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             ss = fmaf(s[k][e], s[k][e], ss);
-        if (live[k])
+        if (live[k] && has_res)
             st_stream(rr + 8 * (v0 + threadIdx.x + k * blockDim.x), packed);
     }
     return ss;
 }
 
-template <int VPT>
+// out = s * inv_rms * gamma: bf16, or (FP8) the E4M3 code of out / scale
+// (round to nearest even, saturated to +-448: cvt.rn.satfinite.e4m3x2.f32).
+template <int VPT, bool FP8>
 __device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int v0,
                                             float inv_rms, float (&s)[VPT][8],
                                             const bool (&live)[VPT])
 {
-    __nv_bfloat16 *orow = p.out + row * p.os;
+    float scale = 1.f;
+    if (FP8)
+        scale = __ldg(p.scale);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         if (!live[k])
@@ -103,12 +105,24 @@ __device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             s[k][e] = (s[k][e] * inv_rms) * g[e];
-        st_stream(orow + 8 * v, pack8(s[k]));
+        if (FP8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 q = make_float2(__fdiv_rn(s[k][2 * i], scale),
+                                             __fdiv_rn(s[k][2 * i + 1], scale));
+                w[i] = (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+            }
+            const uint2 codes = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+            __stcs(reinterpret_cast<uint2 *>(p.out8 + row * p.os + 8 * v), codes);
+        } else {
+            st_stream(p.out + row * p.os + 8 * v, pack8(s[k]));
+        }
     }
 }
 
 // One CTA per row.
-template <int VPT>
+template <int VPT, bool FP8>
 __global__ void __launch_bounds__(kMaxThreads) rms_rows_kernel(const __grid_constant__ RmsParams p)
 {
     pdl_wait();
@@ -120,11 +134,11 @@ __global__ void __launch_bounds__(kMaxThreads) rms_rows_kernel(const __grid_cons
     const float ss = load_sum<VPT>(p, row, 0, p.hidden >> 3, s, live);
     const float total = block_sum(ss, red);
     const float inv_rms = rsqrtf(fmaf(total, p.inv_hidden, p.eps));
-    scale_store<VPT>(p, row, 0, inv_rms, s, live);
+    scale_store<VPT, FP8>(p, row, 0, inv_rms, s, live);
 }
 
 // One cluster per row; CTA `rank` owns vectors [rank*per, (rank+1)*per).
-template <int VPT>
+template <int VPT, bool FP8>
 __global__ void __launch_bounds__(kMaxThreads)
 rms_cluster_kernel(const __grid_constant__ RmsParams p)
 {
@@ -153,30 +167,32 @@ rms_cluster_kernel(const __grid_constant__ RmsParams p)
         total += *cluster.map_shared_rank(&partial, r);
     cluster.barrier_arrive();  // done reading the other CTAs' shared memory
     const float inv_rms = rsqrtf(fmaf(total, p.inv_hidden, p.eps));
-    scale_store<VPT>(p, row, v0, inv_rms, s, live);
+    scale_store<VPT, FP8>(p, row, v0, inv_rms, s, live);
     cluster.barrier_wait();    // no CTA leaves while its partial may still be read
 }
 
 using Fn = void (*)(RmsParams);
 
+template <bool FP8>
 Fn rows_fn(int vpt)
 {
     switch (vpt) {
-    case 1: return rms_rows_kernel<1>;
-    case 2: return rms_rows_kernel<2>;
-    case 4: return rms_rows_kernel<4>;
-    case 8: return rms_rows_kernel<8>;
+    case 1: return rms_rows_kernel<1, FP8>;
+    case 2: return rms_rows_kernel<2, FP8>;
+    case 4: return rms_rows_kernel<4, FP8>;
+    case 8: return rms_rows_kernel<8, FP8>;
     default: return nullptr;
     }
 }
 
+template <bool FP8>
 Fn cluster_fn(int vpt)
 {
     switch (vpt) {
-    case 1: return rms_cluster_kernel<1>;
-    case 2: return rms_cluster_kernel<2>;
-    case 4: return rms_cluster_kernel<4>;
-    case 8: return rms_cluster_kernel<8>;
+    case 1: return rms_cluster_kernel<1, FP8>;
+    case 2: return rms_cluster_kernel<2, FP8>;
+    case 4: return rms_cluster_kernel<4, FP8>;
+    case 8: return rms_cluster_kernel<8, FP8>;
     default: return nullptr;
     }
 }
@@ -207,6 +223,7 @@ void shape(int vectors, int target, int &vpt, int &threads)
 
 cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, LaunchRecord *rec)
 {
+    const bool fp8 = p.out8 != nullptr;
     const int nvec = p.hidden >> 3;
     const int target_ctas = 2 * sm_count();
     int cs = 1;
@@ -225,9 +242,10 @@ cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, La
 
     cudaError_t err;
     if (cs == 1) {
-        err = launch(rows_fn(vpt), dim3((unsigned)grid), dim3(threads), 0, stream, 1, p);
+        err = launch(fp8 ? rows_fn<true>(vpt) : rows_fn<false>(vpt), dim3((unsigned)grid),
+                     dim3(threads), 0, stream, 1, p);
     } else {
-        Fn fn = cluster_fn(vpt);
+        Fn fn = fp8 ? cluster_fn<true>(vpt) : cluster_fn<false>(vpt);
         if (cs > 8) {
             err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (err != cudaSuccess)

@@ -68,6 +68,13 @@ def _load():
         lib.oracle_vit_planes.argtypes = [P, I64, P, I64, P, I64, P, I64, P, P, P]
         lib.oracle_rms_norm_residual.restype = None
         lib.oracle_rms_norm_residual.argtypes = [P, P, P, I64, I64, ctypes.c_double, P, P]
+        lib.oracle_fp8_e4m3.restype = ctypes.c_uint8
+        lib.oracle_fp8_e4m3.argtypes = [ctypes.c_double]
+        lib.oracle_fp8_e4m3_array.restype = None
+        lib.oracle_fp8_e4m3_array.argtypes = [P, I64, P]
+        lib.oracle_rms_norm_fp8.restype = None
+        lib.oracle_rms_norm_fp8.argtypes = [P, P, P, I64, I64, ctypes.c_double, ctypes.c_double,
+                                            P, P, P]
         _lib = lib
     return _lib
 
@@ -224,3 +231,26 @@ def rms_norm_residual(x, residual, gamma, eps: float):
     lib.oracle_rms_norm_residual(_ptr(xb), _ptr(rb), _ptr(gb), R, hidden, float(eps),
                                  _ptr(res_out), _ptr(out))
     return res_out, out
+
+
+def fp8_e4m3(values) -> np.ndarray:
+    """E4M3 ("FN") codes of fp64 values: round to nearest even, saturate at 448."""
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float64))
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().oracle_fp8_e4m3_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def rms_norm_fp8(x, residual, gamma, eps: float, scale: float):
+    """(new residual bf16 bits or None, y / scale in fp64, E4M3 codes), [R, hidden]."""
+    lib = _load()
+    xb, gb = bits(x), bits(gamma)
+    R, hidden = xb.shape
+    rb = bits(residual) if residual is not None else None
+    res_out = np.empty((R, hidden), dtype=np.uint16)
+    ys = np.empty((R, hidden), dtype=np.float64)
+    codes = np.empty((R, hidden), dtype=np.uint8)
+    lib.oracle_rms_norm_fp8(_ptr(xb), _ptr(rb) if rb is not None else None, _ptr(gb), R,
+                            hidden, float(eps), float(scale), _ptr(res_out), _ptr(ys),
+                            _ptr(codes))
+    return (res_out if rb is not None else None), ys, codes

@@ -350,3 +350,81 @@ void oracle_rms_norm_residual(const uint16_t *x, const uint16_t *res, const uint
             out[r * hidden + i] = bf16_value(ro[i]) * inv_rms * bf16_value(gamma[i]);
     }
 }
+
+/* ------------------------------------------------------ FP8 E4M3 encoding -- */
+/*
+ * The static-FP8 output of rms_norm_fp8 (vLLM #26234 names the fused
+ * rms_norm_static_fp8_quant_kernel; the format is the OCP FP8 E4M3 "FN" one
+ * that kernel family writes): 1 sign bit, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent field 0 holds the subnormals m * 2^-9; there are no
+ * infinities and S.1111.111 is NaN, so the largest finite magnitude is
+ * 1.75 * 2^8 = 448.  Values are rounded to the nearest representable value,
+ * ties to the even mantissa, and magnitudes above 448 saturate to 448.
+ */
+uint8_t oracle_fp8_e4m3(double v)
+{
+    if (isnan(v))
+        return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    unsigned code;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal grid: steps of 2^-9; a rounding up to 8 steps is the
+         * smallest normal, whose code is 8 as well */
+        code = (unsigned)nearbyint(a * 512.0);
+    } else {
+        int e;
+        frexp(a, &e);          /* a = f * 2^e, f in [0.5, 1) */
+        e -= 1;                /* a = g * 2^e, g in [1, 2) */
+        double q = nearbyint(ldexp(a, 3 - e));   /* g * 8 rounded: 8 .. 16 */
+        if (q >= 16.0) {
+            q = 8.0;
+            e += 1;
+        }
+        if (e + 7 > 15)
+            return sign | 0x7E;
+        code = ((unsigned)(e + 7) << 3) | ((unsigned)q - 8u);
+    }
+    if (code > 0x7E)
+        code = 0x7E;
+    return sign | (uint8_t)code;
+}
+
+void oracle_fp8_e4m3_array(const double *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_fp8_e4m3(v[i]);
+}
+
+/*
+ * rms_norm_fp8: with a residual (res != NULL) s = bf16(x + residual) becomes
+ * the new residual; without one s = x.  y = s / sqrt(mean(s^2) + eps) * gamma
+ * in fp64; y_scaled = y / scale; codes = E4M3(y_scaled).
+ */
+void oracle_rms_norm_fp8(const uint16_t *x, const uint16_t *res, const uint16_t *gamma,
+                         int64_t R, int64_t hidden, double eps, double scale,
+                         uint16_t *res_out, double *y_scaled, uint8_t *codes)
+{
+    for (int64_t r = 0; r < R; ++r) {
+        const uint16_t *xr = x + r * hidden;
+        double ss = 0.0;
+        for (int64_t i = 0; i < hidden; ++i) {
+            double s;
+            if (res) {
+                res_out[r * hidden + i] =
+                    oracle_bf16_round(bf16_value(xr[i]) + bf16_value(res[r * hidden + i]));
+                s = bf16_value(res_out[r * hidden + i]);
+            } else {
+                s = bf16_value(xr[i]);
+            }
+            ss += s * s;
+        }
+        double inv_rms = 1.0 / sqrt(ss / (double)hidden + eps);
+        for (int64_t i = 0; i < hidden; ++i) {
+            double s = res ? bf16_value(res_out[r * hidden + i]) : bf16_value(xr[i]);
+            double y = s * inv_rms * bf16_value(gamma[i]);
+            y_scaled[r * hidden + i] = y / scale;
+            codes[r * hidden + i] = oracle_fp8_e4m3(y / scale);
+        }
+    }
+}

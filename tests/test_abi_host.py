@@ -230,3 +230,21 @@ def test_rope_set_rows_refusals(qkr):
     assert call(flags=qkr.FLAG_ROUND_NORMALIZED_BF16) == E  # rounding contract needs gamma
     assert call(T=0, rows=None) == qkr.QKR_OK           # empty: nothing enqueued
     assert qkr.last_launch()["launches"] == 0
+
+
+def test_rms_norm_fp8_refusals(qkr):
+    E, U = qkr.QKR_ERR_INVALID_ARG, qkr.QKR_ERR_UNSUPPORTED
+    L = qkr.lib()
+
+    def call(x=FAKE, res=FAKE + (1 << 20), gamma=FAKE + (2 << 20), out=FAKE + (3 << 20),
+             scale=FAKE + (4 << 20), R=4, hidden=64, xs=64, rs=64, os=64):
+        return L.rms_norm_fp8(None, x, res, gamma, out, scale, R, hidden, xs, rs, os, 1e-6)
+    assert call(scale=None) == E                 # the static scale is required
+    assert call(out=FAKE + (3 << 20) + 4) == U   # FP8 rows need 8-byte alignment
+    assert call(os=60) == U                      # stride below hidden
+    assert call(out=FAKE + 64) == U              # out overlaps x
+    assert call(scale=FAKE + (1 << 20) + 8) == U  # scale inside the residual it rewrites
+    assert call(scale=FAKE + (3 << 20) + 8) == U  # scale inside out
+    assert call(hidden=60, xs=60, rs=60, os=60) == U
+    assert call(R=0) == qkr.QKR_OK
+    assert qkr.last_launch()["launches"] == 0

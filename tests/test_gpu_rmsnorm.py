@@ -94,3 +94,61 @@ def test_deterministic_repeat():
     _, o1 = run_rms(w)
     _, o2 = run_rms(w)
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+def _decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(codes.astype(np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def assert_fp8_codes(got: np.ndarray, ref_vals: np.ndarray, ref_codes: np.ndarray, what=""):
+    """Codes must equal the oracle's, except where the oracle's exact value
+    lies within 1e-5 (relative) of the midpoint between the oracle's code and
+    an adjacent one (the GPU takes the rounding decision from its fp32 value,
+    which differs from the fp64 value by a few fp32 ulps); those few may take
+    the neighbour."""
+    bad = got != ref_codes
+    if not bad.any():
+        return 0
+    gv = _decode_e4m3(got[bad])
+    rv = _decode_e4m3(ref_codes[bad])
+    v = ref_vals[bad]
+    mid = 0.5 * (gv + rv)
+    near = np.abs(v - mid) <= 1e-5 * np.abs(mid) + 1e-12
+    # adjacent: no representable value strictly between the two codes
+    adjacent = np.abs(got[bad].astype(int) - ref_codes[bad].astype(int)) == 1
+    ok = near & adjacent
+    assert ok.all(), "%s: %d codes differ beyond a rounding tie; first got %s ref %s value %r" % (
+        what, int((~ok).sum()), hex(int(got[bad][~ok][0])), hex(int(ref_codes[bad][~ok][0])),
+        float(v[~ok][0]))
+    assert bad.sum() <= max(2, 1e-4 * got.size), "%s: too many tie flips" % what
+    return int(bad.sum())
+
+
+@pytest.mark.parametrize("R,hidden,with_res,scale", [
+    (1, 5120, True, 0.05), (32, 5120, True, 0.05), (1000, 2048, True, 1.0),
+    (3, 8192, False, 0.02), (257, 4096, False, 0.5), (64, 2048, True, 1e-3)])
+def test_rms_norm_fp8_vs_oracle(R, hidden, with_res, scale):
+    w = W.config2(R=R, hidden=hidden, seed=600 + R)
+    x = to_dev(w.x)
+    res = None
+    if with_res:
+        res_g = Guarded(w.residual.shape)
+        res_g.tensor.copy_(to_dev(w.residual))
+        res = res_g.tensor
+    guard = 4096
+    buf = torch.full((guard + R * hidden + guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    out8 = buf[guard:guard + R * hidden].view(R, hidden)
+    sc = torch.tensor([scale], dtype=torch.float32, device="cuda")
+    qkr.rms_norm_fp8(x, res, to_dev(w.gamma), out8, sc, w.eps)
+    torch.cuda.synchronize()
+    assert bool((buf[:guard] == 0xA5).all()) and bool((buf[guard + R * hidden:] == 0xA5).all()), \
+        "write outside the FP8 output"
+    info = qkr.last_launch()
+    assert info["kernel_name"] in ("rms_rows", "rms_cluster")
+    ref_res, ys, codes = oracle.rms_norm_fp8(w.x, w.residual if with_res else None, w.gamma,
+                                             w.eps, scale)
+    if with_res:
+        res_g.check()
+        assert np.array_equal(oracle.bits(res), ref_res), "residual stream not bit-exact"
+    got = out8.cpu().numpy()
+    assert_fp8_codes(got, ys, codes, "R=%d hidden=%d" % (R, hidden))

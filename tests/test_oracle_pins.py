@@ -557,3 +557,60 @@ def test_scatter_rows_places_each_row_once():
         assert (out[r] == -1.0).all()
     rev = oracle.scatter_rows(rows, [3, 2, 1, 0], 4)
     assert np.array_equal(rev, rows[::-1])
+
+
+def _e4m3_decode(code: int) -> float:
+    """The E4M3 ("FN") format written out: sign, 4-bit exponent (bias 7),
+    3-bit mantissa, exponent 0 = subnormal m * 2^-9."""
+    s = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 7
+    if e == 0:
+        return s * m * 2.0 ** -9
+    return s * (1 + m / 8) * 2.0 ** (e - 7)
+
+
+def test_fp8_e4m3_hand_values():
+    cases = [(1.0, 0x38), (3.5, 0x46), (-3.5, 0xC6), (448.0, 0x7E), (-448.0, 0xFE),
+             (2.0 ** -9, 0x01), (7 * 2.0 ** -9, 0x07), (2.0 ** -6, 0x08),
+             (2.0 ** -10, 0x00),              # tie between 0 and the smallest subnormal: even
+             (3 * 2.0 ** -10, 0x02),          # tie between 1 and 2 subnormal steps: even
+             (1.0625, 0x38), (1.1875, 0x3A),  # ties between mantissas 0/1 and 1/2
+             (464.0, 0x7E), (470.0, 0x7E), (500.0, 0x7E), (-1e9, 0xFE),  # saturation
+             (0.0, 0x00), (-0.0, 0x80)]
+    for v, code in cases:
+        assert int(oracle.fp8_e4m3([v])[0]) == code, (v, hex(code))
+
+
+def test_fp8_e4m3_round_trip_and_torch():
+    """Every finite code decodes (format definition above; torch's own
+    float8_e4m3fn agrees) and re-encodes to itself; random values in range
+    encode as torch's round-to-nearest-even cast does."""
+    codes = [c for c in range(256) if (c & 0x7F) != 0x7F]
+    vals = np.array([_e4m3_decode(c) for c in codes])
+    t = torch.tensor(codes, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(vals, t)
+    enc = oracle.fp8_e4m3(vals)
+    assert np.array_equal(enc[vals != 0], np.array(codes, dtype=np.uint8)[vals != 0])
+    rng = np.random.default_rng(3)
+    r = np.concatenate([rng.uniform(-448, 448, 4000), rng.normal(0, 0.05, 4000),
+                        rng.normal(0, 2 ** -8, 2000)])
+    want = torch.from_numpy(r).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.fp8_e4m3(r), want)
+
+
+def test_rms_norm_fp8_matches_rms_norm_and_encoder():
+    """The FP8 RMSNorm is the bf16-path RMSNorm divided by the scale and
+    encoded: same residual bits, y/scale equals out/scale, codes equal the
+    encoder's; without a residual s = x."""
+    w = W.config2(R=3, hidden=64, seed=41)
+    res_o, y_o = oracle.rms_norm_residual(w.x, w.residual, w.gamma, w.eps)
+    res_f, ys, codes = oracle.rms_norm_fp8(w.x, w.residual, w.gamma, w.eps, 0.05)
+    assert np.array_equal(res_o, res_f)
+    assert np.allclose(ys, y_o / 0.05, rtol=1e-15, atol=0)
+    assert np.array_equal(codes, oracle.fp8_e4m3(ys))
+    zero = torch.zeros_like(w.residual)
+    _, y_z = oracle.rms_norm_residual(w.x, zero, w.gamma, w.eps)
+    none, ys_n, _ = oracle.rms_norm_fp8(w.x, None, w.gamma, w.eps, 2.0)
+    assert none is None
+    assert np.allclose(ys_n, y_z / 2.0, rtol=1e-15, atol=0)
