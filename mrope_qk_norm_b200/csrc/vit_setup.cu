@@ -3,11 +3,14 @@
 // expose the section rule and the grid-to-position mapping to the tests.
 //
 // B200 mapping.  The setup writes 2 * 4 bytes per (token, section column),
-// computing one sincosf per cell; it is store-bound at large N and
-// launch-bound at small N.  A CTA covers kTokens tokens: one thread per token
-// derives (t, h, w) once into shared memory, then all threads walk the
-// tokens' (token, column) cells with consecutive threads on consecutive
-// columns, so each warp's stores fall into a few contiguous runs of a plane.
+// computing one sincosf per cell; it is latency- and launch-bound at these
+// sizes (8 MB for 16k tokens).  A CTA covers kTokens tokens.  It first stages
+// the grid metadata (cu_seqlens, grids) and inv_freq in shared memory with
+// independent loads -- one memory round trip instead of the binary search's
+// chain of dependent loads -- then one thread per token derives (t, h, w)
+// into shared memory, and each thread keeps one column (axis, offset and
+// inv_freq fixed in registers) while walking the tokens, consecutive threads
+// on consecutive columns so each warp's stores are contiguous.
 
 #include <climits>
 
@@ -18,8 +21,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTokens = 32;
+constexpr int kSmemGrids = 512;  // grids whose metadata a CTA stages in shared memory
+constexpr int kMaxVitPairs = 512;  // per-axis inv_freq lengths staged in shared memory
 
-// (t, h, w) of token n.  The grid is the g with cu[g] <= n < cu[g+1]
+// (t, h, w) of token n (cu / grids in shared or global memory).  The grid is
+// the g with cu[g] <= n < cu[g+1]
 // (binary search over the nondecreasing boundaries; empty grids are never
 // selected).  Inside a frame of h*w tokens, tokens come in m x m merge blocks
 // in row-major block order, each block's patches in row-major order.
@@ -29,15 +35,15 @@ __device__ __forceinline__ void token_position(const int32_t *cu, const int32_t 
     int lo = 0, hi = G;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if ((int64_t)__ldg(cu + mid + 1) <= n)
+        if ((int64_t)cu[mid + 1] <= n)
             lo = mid + 1;
         else
             hi = mid;
     }
     const int g = lo < G ? lo : G - 1;
-    const int64_t local = n - (int64_t)__ldg(cu + g);
-    const int h = __ldg(grids + 3 * g + 1);
-    const int w = __ldg(grids + 3 * g + 2);
+    const int64_t local = n - (int64_t)cu[g];
+    const int h = grids[3 * g + 1];
+    const int w = grids[3 * g + 2];
     const int64_t frame = max((int64_t)h * w, (int64_t)1);
     tp = (int)(local / frame);
     const int64_t in_frame = local - (int64_t)tp * frame;
@@ -56,11 +62,32 @@ __global__ void __launch_bounds__(kThreads) vit_setup_kernel(const __grid_consta
     pdl_wait();
     pdl_trigger();
     __shared__ int spos[3][kTokens];
+    __shared__ int32_t scu[kSmemGrids + 1];
+    __shared__ int32_t sgrid[3 * kSmemGrids];
+    __shared__ float sinv[3][kMaxVitPairs];
+    // Stage the grid metadata and inv_freq with independent loads (one DRAM
+    // round trip) instead of the binary search's chain of dependent loads.
+    const bool staged = p.G <= kSmemGrids;
+    if (staged) {
+        for (int i = threadIdx.x; i <= p.G; i += kThreads)
+            scu[i] = __ldg(p.cu + i);
+        for (int i = threadIdx.x; i < 3 * p.G; i += kThreads)
+            sgrid[i] = __ldg(p.grids + i);
+    }
+    const bool inv_staged =
+        p.half[0] <= kMaxVitPairs && p.half[1] <= kMaxVitPairs && p.half[2] <= kMaxVitPairs;
+    if (inv_staged)
+        for (int a = 0; a < 3; ++a)
+            for (int i = threadIdx.x; i < p.half[a]; i += kThreads)
+                sinv[a][i] = __ldg(p.inv[a] + i);
+    __syncthreads();
+
     const int64_t n0 = (int64_t)blockIdx.x * kTokens;
     const int ntok = (int)min((int64_t)kTokens, p.N - n0);
     if (threadIdx.x < ntok) {
         int tp, hp, wp;
-        token_position(p.cu, p.grids, p.G, n0 + threadIdx.x, p.m, tp, hp, wp);
+        token_position(staged ? scu : p.cu, staged ? sgrid : p.grids, p.G, n0 + threadIdx.x,
+                       p.m, tp, hp, wp);
         spos[0][threadIdx.x] = tp;
         spos[1][threadIdx.x] = hp;
         spos[2][threadIdx.x] = wp;
@@ -69,17 +96,42 @@ __global__ void __launch_bounds__(kThreads) vit_setup_kernel(const __grid_consta
 
     const int P = p.P;
     const int end_t = p.half[0], end_h = p.half[0] + p.half[1];
-    for (int idx = threadIdx.x; idx < ntok * P; idx += kThreads) {
-        const int tt = idx / P;
-        const int col = idx - tt * P;
-        const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
-        const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
-        const float theta = __fmul_rn((float)spos[axis][tt], __ldg(p.inv[axis] + (col - off)));
-        float s, c;
-        sincosf(theta, &s, &c);
-        const int64_t at = ((int64_t)axis * p.N + n0 + tt) * P + col;
-        p.cos_out[at] = c;
-        p.sin_out[at] = s;
+    if (P <= kThreads) {
+        // A thread owns one column for the whole pass: its axis, section
+        // offset and inv_freq are fixed, and it walks the CTA's tokens with
+        // a stride of kThreads / P (consecutive threads on consecutive
+        // columns of one token row, so each warp's stores are contiguous).
+        const int tpp = kThreads / P;
+        const int col = threadIdx.x % P;
+        const int tsub = threadIdx.x / P;
+        if (tsub < tpp) {
+            const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
+            const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
+            const float f = inv_staged ? sinv[axis][col - off] : __ldg(p.inv[axis] + (col - off));
+            const int64_t base = ((int64_t)axis * p.N + n0) * P + col;
+#pragma unroll 4
+            for (int tt = tsub; tt < ntok; tt += tpp) {
+                const float theta = __fmul_rn((float)spos[axis][tt], f);
+                float s, c;
+                sincosf(theta, &s, &c);
+                __stcs(p.cos_out + base + (int64_t)tt * P, c);
+                __stcs(p.sin_out + base + (int64_t)tt * P, s);
+            }
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < ntok * P; idx += kThreads) {
+            const int tt = idx / P;
+            const int col = idx - tt * P;
+            const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
+            const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
+            const float f = inv_staged ? sinv[axis][col - off] : __ldg(p.inv[axis] + (col - off));
+            const float theta = __fmul_rn((float)spos[axis][tt], f);
+            float s, c;
+            sincosf(theta, &s, &c);
+            const int64_t at = ((int64_t)axis * p.N + n0 + tt) * P + col;
+            __stcs(p.cos_out + at, c);
+            __stcs(p.sin_out + at, s);
+        }
     }
 }
 

@@ -78,6 +78,23 @@ def test_setup_odd_lengths_and_single_grid():
     assert np.array_equal(cos.untouched(), ~mask)
 
 
+def test_setup_many_grids_and_long_axis():
+    """More grids than a CTA stages in shared memory (600 > 512) and an axis
+    longer than the staged inv_freq (600 > 512): the kernel reads that
+    metadata from global memory instead, with the same results."""
+    rng = np.random.default_rng(53)
+    grids = [[int(rng.integers(1, 3)), 2 * int(rng.integers(1, 3)), 2 * int(rng.integers(1, 3))]
+             for _ in range(600)]
+    w = W.config5(seed=53, grids=grids, lens=(3, 600, 5), spatial_merge=2)
+    cos, sin, _, _, _ = run_setup(w)
+    pos = oracle.vit_positions(w.grids, 2)
+    rc, rs, written = oracle.vit_planes(pos, w.inv_t, w.inv_h, w.inv_w)
+    mask = written.astype(bool)
+    assert_plane_close(cos.tensor.cpu().numpy(), rc, mask, "cos")
+    assert_plane_close(sin.tensor.cpu().numpy(), rs, mask, "sin")
+    assert np.array_equal(cos.untouched(), ~mask)
+
+
 def test_setup_empty_grid_list():
     inv = torch.ones(4, dtype=torch.float32, device="cuda")
     e32 = torch.empty(0, dtype=torch.int32, device="cuda")
