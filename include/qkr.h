@@ -324,7 +324,8 @@ qkr_status rms_norm_residual(void *stream, const void *x, void *residual, const 
  * is written back to residual as in rms_norm_residual; without one
  * (residual == NULL) s = x.  Then y = s * rsqrt(mean(s^2) + eps) * gamma in
  * fp32, and out holds the FP8 E4M3 (OCP "FN": no infinities, max 448) code of
- * y / scale, rounded to nearest even and saturated to +-448.
+ * y / scale (computed as y * fp32(1 / scale)), rounded to nearest even and
+ * saturated to +-448.
  *
  *   out              device uint8 [R, hidden] E4M3 codes, row stride out_stride
  *                    bytes (a multiple of 8), 8-byte aligned.
@@ -407,6 +408,14 @@ qkr_status qkr_launch_overlap(int32_t enable);
  * range. */
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,
                          int32_t stages);
+
+/* Lanes sharing one head row in the GPT-J (VECTOR) layout of the rope
+ * kernels, for tuning sweeps: 0 automatic, else 1, 2, 4, 8 or 16 (ignored
+ * where a lane would need more than two 16-byte vectors of the row).
+ * Process-wide.  The lane count sets the order of the fp32 sum of squares
+ * (per-lane partial sums, then a shuffle tree), so results can differ in the
+ * last bit between choices; each choice is deterministic. */
+qkr_status qkr_tune_rope_lanes(int32_t lanes);
 
 /* Device status word of the library on the current device (0 = healthy).
  * Kernels that wait on shared-memory barriers give every wait a time budget;

@@ -29,7 +29,8 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
 
 EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "rope_set_rows",
            "vit_mrope_setup", "rms_norm_residual", "rms_norm_fp8", "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
-           "qkr_vit_positions", "qkr_tune_rope", "qkr_device_status", "qkr_launch_overlap")
+           "qkr_vit_positions", "qkr_tune_rope", "qkr_tune_rope_lanes", "qkr_device_status",
+           "qkr_launch_overlap")
 
 
 class QkrError(RuntimeError):
@@ -92,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "qkr_section_map": [V, I32, V, I64, V],
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
         "qkr_tune_rope": [I32, I32, I32, I32],
+        "qkr_tune_rope_lanes": [I32],
         "qkr_launch_overlap": [I32],
         "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
     }
@@ -164,6 +166,11 @@ def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 
     """Override the rope kernels' launch shape (0 = automatic), for tuning.
     pipeline: 1 item kernel, 2 bulk-copy pipelined kernel, 3 streaming kernel."""
     _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta, stages))
+
+
+def tune_rope_lanes(lanes: int = 0) -> None:
+    """Lanes per head row of the GPT-J layout (0 = automatic), for tuning."""
+    _check(_lib.qkr_tune_rope_lanes(lanes))
 
 
 def launch_overlap(enable: bool) -> None:

@@ -445,6 +445,15 @@ qkr_status qkr_launch_overlap(int32_t enable)
     return QKR_OK;
 }
 
+qkr_status qkr_tune_rope_lanes(int32_t lanes)
+{
+    if (lanes != 0 && lanes != 1 && lanes != 2 && lanes != 4 && lanes != 8 && lanes != 16)
+        return fail(QKR_ERR_INVALID_ARG, "lanes must be 0 or a power of two up to 16");
+    qkr::set_rope_lanes_override(lanes);
+    g_error.clear();
+    return QKR_OK;
+}
+
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,
                          int32_t stages)
 {

@@ -193,6 +193,8 @@ struct LaunchRecord {
 // 1 register kernel only, 2 bulk-copy pipelined kernel only.
 void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta,
                              int stages);
+// Lanes per head row of the GPT-J (VECTOR) layout, for tuning (0: automatic).
+void set_rope_lanes_override(int lanes);
 
 // Bulk-copy pipelined rope kernel (rope_tma.cu); cudaErrorNotSupported when a
 // call is outside what it serves.

@@ -85,16 +85,18 @@ __device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v
     return ss;
 }
 
-// out = s * inv_rms * gamma: bf16, or (FP8) the E4M3 code of out / scale
-// (round to nearest even, saturated to +-448: cvt.rn.satfinite.e4m3x2.f32).
+// out = s * inv_rms * gamma: bf16, or (FP8) the E4M3 code of out / scale,
+// computed as out * fp32(1 / scale) (one multiply per element instead of a
+// division), rounded to nearest even and saturated to +-448
+// (cvt.rn.satfinite.e4m3x2.f32).
 template <int VPT, bool FP8>
 __device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int v0,
                                             float inv_rms, float (&s)[VPT][8],
                                             const bool (&live)[VPT])
 {
-    float scale = 1.f;
+    float inv_scale = 1.f;  // y / scale is taken as y * fp32(1 / scale)
     if (FP8)
-        scale = __ldg(p.scale);
+        inv_scale = __frcp_rn(__ldg(p.scale));
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         if (!live[k])
@@ -109,8 +111,8 @@ __device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float2 q = make_float2(__fdiv_rn(s[k][2 * i], scale),
-                                             __fdiv_rn(s[k][2 * i + 1], scale));
+                const float2 q = make_float2(s[k][2 * i] * inv_scale,
+                                             s[k][2 * i + 1] * inv_scale);
                 w[i] = (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
             }
             const uint2 codes = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
