@@ -141,15 +141,36 @@ struct Item {
     bool s1;                   // second stream
 };
 
+// Position of a lane group in the CTA's item sequence (item = tt * gpt + b),
+// advanced by G items per pass without an integer division.
+struct ItemCursor {
+    int tt;  // token within the CTA's range
+    int b;   // item within the token, [0, gpt)
+    __device__ __forceinline__ void start(int item, int gpt)
+    {
+        tt = item / gpt;
+        b = item - tt * gpt;
+    }
+    // dq = G / gpt, dr = G % gpt
+    __device__ __forceinline__ void advance(int dq, int dr, int gpt)
+    {
+        tt += dq;
+        b += dr;
+        if (b >= gpt) {
+            b -= gpt;
+            ++tt;
+        }
+    }
+};
+
 template <int U>
-__device__ __forceinline__ Item decode_item(const RopeParams &p, int64_t tok0, int item,
-                                            int items, int gpt, int nbq)
+__device__ __forceinline__ Item decode_item(const RopeParams &p, int64_t tok0,
+                                            const ItemCursor &c, int ntok, int nbq)
 {
     Item r;
-    const bool live = item < items;
-    const int it = live ? item : 0;
-    r.tt = it / gpt;
-    const int b = it - r.tt * gpt;
+    const bool live = c.tt < ntok;
+    r.tt = live ? c.tt : 0;
+    const int b = live ? c.b : 0;
     r.isk = b >= nbq;
     const int h0 = (r.isk ? b - nbq : b) * U;
     r.nh = live ? min(U, (r.isk ? p.Hk : p.Hq) - h0) : 0;
@@ -275,8 +296,11 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
     const int gpt = nbq + (p.Hk + U - 1) / U;
     const int items = ntok * gpt;
 
-    for (int it0 = 0; it0 < items; it0 += G) {  // uniform trip count across the CTA
-        const Item m = decode_item<U>(p, tok0, it0 + grp, items, gpt, nbq);
+    ItemCursor cur;
+    cur.start(grp, gpt);
+    const int dq = G / gpt, dr = G - (G / gpt) * gpt;
+    for (int it0 = 0; it0 < items; it0 += G, cur.advance(dq, dr, gpt)) {  // uniform trips
+        const Item m = decode_item<U>(p, tok0, cur, ntok, nbq);
 
         uint4 raw[U][NS];
 #pragma unroll

@@ -114,9 +114,14 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
 
     // Copy this thread's vectors of pass `pass` into ring stage `pass % S`
     // (one commit group per pass, empty past the last pass).
+    const int dq = G / gpt, dr = G - (G / gpt) * gpt;
+    ItemCursor icur, ccur;  // the pass being copied in, the pass being computed
+    icur.start(grp, gpt);
+    ccur = icur;
     auto issue = [&](int pass) {
         if (pass < passes) {
-            const Item m = decode_item<U>(p, tok0, pass * G + grp, items, gpt, nbq);
+            const Item m = decode_item<U>(p, tok0, icur, ntok, nbq);
+            icur.advance(dq, dr, gpt);
             const int st = pass % S;
 #pragma unroll
             for (int u = 0; u < U; ++u)
@@ -138,7 +143,8 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     for (int pass = 0; pass < passes; ++pass) {
         issue(pass + S - 1);
         cp_async_wait(S - 1);
-        const Item m = decode_item<U>(p, tok0, pass * G + grp, items, gpt, nbq);
+        const Item m = decode_item<U>(p, tok0, ccur, ntok, nbq);
+        ccur.advance(dq, dr, gpt);
         const int st = pass % S;
 
         float2 C[NQ], Sn[NQ];
