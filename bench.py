@@ -467,6 +467,46 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
                       % (calls, tokens, N_IMG_SAMPLE, dt)}
 
 
+def cpu_baseline_parallel(budget_s: float = 8.0) -> dict:
+    """The same oracle run concurrently on every host core the process may use:
+    thread i repeatedly processes its own slice of the image stream (the
+    oracle is C called through ctypes, which releases the GIL)."""
+    import concurrent.futures
+    import oracle
+    cores = max(1, min(len(os.sched_getaffinity(0)), 64))
+    w = W.config3()
+    img = w.streams[1]
+    T_txt = w.streams[0].q.shape[0]
+    T_img = img.q.shape[0]
+    per = max(1, T_img // cores)
+    slices = []
+    for i in range(cores):
+        a = (i * per) % T_img
+        b = min(a + per, T_img)
+        s = W.StreamInputs(img.q[a:b], img.k[a:b], img.gamma_q, img.gamma_k)
+        ang = W.AngleInputs(kind=w.angle.kind, cos=w.angle.cos, sin=w.angle.sin,
+                            token_offset=T_txt + a)
+        slices.append((s, ang, b - a))
+    oracle.build()
+    t_end = time.perf_counter() + budget_s
+
+    def work(i):
+        s, ang, n = slices[i]
+        done = 0
+        while time.perf_counter() < t_end:
+            oracle.qk_norm_rope([s], 24, 24, 128, 128, w.pairing, w.eps, ang)
+            done += n
+        return done
+
+    t0 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=cores) as ex:
+        total = sum(ex.map(work, range(cores)))
+    dt = time.perf_counter() - t0
+    return {"value": round(total / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d threads, each repeating the oracle on its own %d-token slice of the "
+                      "headline's image stream, %.1f s" % (cores, per, dt)}
+
+
 def reference_arm(args) -> dict:
     """The CPU oracle timed like our arm: W untimed steps, then K timed steps,
     each step one oracle call on the bounded sample."""
@@ -639,9 +679,10 @@ def main():
     if not args.no_rows and not args.no_rms_sweep and world == 1:
         sweep = rms_sweep(dev, stream, peaks["hbm_gbs"])
 
-    cb = None
+    cb = cbp = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cb = cpu_baseline()
+        cbp = cpu_baseline_parallel()
 
     if dist:
         dist.barrier()
@@ -677,6 +718,7 @@ def main():
                      "frac_of_same_size_elementwise": round(copy_us / (kern_ms * 1e3), 4),
                      "kernel": info.get("kernel_name")},
         "cpu_baseline": cb,
+        "cpu_baseline_all_cores": cbp,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "path": "pinned host -> cudaMemcpyAsync -> fused_qk_norm_rope -> pinned host"},
