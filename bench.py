@@ -615,13 +615,11 @@ def main():
     del graph
     info = qkr.last_launch()
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_max = float(t.item())
+    from mrope_qk_norm_b200.sharding import job_tokens_per_s, max_over_ranks
+    total_max = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_max / args.steps
     tokens = w.n_tokens
-    value = world * tokens / (ms_per_step * 1e-3)
+    value = job_tokens_per_s(world, tokens, ms_per_step)
     kern_ms = statistics.mean(per)
     achieved = nbytes / (kern_ms * 1e-3) / 1e9
 
@@ -663,11 +661,8 @@ def main():
             e2e_step()
         e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / args.e2e_steps
-    e2e_value = world * tokens / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.e2e_steps
+    e2e_value = job_tokens_per_s(world, tokens, e2e_ms)
 
     rows = []
     if not args.no_rows:

@@ -70,3 +70,31 @@ def test_two_rank_shards_equal_unsharded(tmp_path):
     port = _free_port()
     mp.spawn(_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
     assert (tmp_path / "result").read_text() == "ok"
+
+
+def _timing_worker(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from mrope_qk_norm_b200.sharding import job_tokens_per_s, max_over_ranks
+        local_ms = [30.0, 42.5][rank]          # the two ranks' own device times
+        slowest = max_over_ranks(local_ms, dist, "cpu")
+        value = job_tokens_per_s(world, 4608, slowest / 2000)
+        with open(os.path.join(out_dir, "rank%d" % rank), "w") as f:
+            f.write("%r %r" % (slowest, value))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_takes_the_slowest_rank(tmp_path):
+    """bench.py's multi-rank aggregation: every rank gets the maximum of the
+    ranks' device times, and whole-job throughput counts all ranks' tokens over
+    that time (weak scaling)."""
+    port = _free_port()
+    mp.spawn(_timing_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    for r in range(2):
+        slowest, value = map(float, (tmp_path / ("rank%d" % r)).read_text().split())
+        assert slowest == 42.5
+        assert abs(value - 2 * 4608 / (42.5 / 2000 * 1e-3)) < 1e-6 * value
