@@ -40,7 +40,7 @@
 // Addresses are 64-bit throughout (large storage offsets, vllm-omni #7600).
 #pragma once
 
-#include "qkr_internal.cuh"
+#include "rope_math.cuh"
 
 namespace qkr {
 
@@ -57,30 +57,6 @@ KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, bool round);
 namespace {
 
 constexpr int kThreads = 256;
-
-enum Layout { PAIRED = 0, VECTOR = 1, EXCHANGE = 2 };
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
-
-__device__ __forceinline__ uint32_t word(const uint4 &v, int i)
-{
-    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
-__device__ __forceinline__ void set_word(uint4 &v, int i, uint32_t w)
-{
-    if (i == 0) v.x = w;
-    else if (i == 1) v.y = w;
-    else if (i == 2) v.z = w;
-    else v.w = w;
-}
-
-__device__ __forceinline__ float2 round2_bf16(float2 a)
-{
-    const uint32_t w = pack2(a.x, a.y);
-    return f2(bf_lo(w), bf_hi(w));
-}
 
 // Stage (cos, sin) of `ntok` tokens into shared memory, SoA, row stride cs_ld.
 // Columns [P, pw) get the identity rotation (1, 0).
@@ -246,8 +222,8 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
     pdl_trigger();
     // Quads (couples of pairs) per lane: PAIRED lo/hi vectors hold 4, each
     // VECTOR slot holds 2.  Pass-through slots (PAIRED tail) are scaled only.
-    constexpr int NQ = LAYOUT == PAIRED ? 4 : 2 * NS;
-    constexpr int NT = LAYOUT == PAIRED ? NS - 2 : 0;
+    constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
+    constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
     constexpr int G = kThreads / LPR;
 
     extern __shared__ float4 smem[];
@@ -335,7 +311,7 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
             }
         }
         // gamma of this lane's columns, in the same (A, B) arrangement
-        float2 GA[NQ], GB[NQ], GT[NT > 0 ? NT : 1][4];
+        float2 GA[NQ], GB[NQ], GT[NTA][4];
         if (NORM) {
             const RopeStreamDev &S = m.s1 ? p.st[1] : p.st[0];
             const __nv_bfloat16 *gam = m.isk ? S.gk : S.gq;
@@ -343,114 +319,26 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
 #pragma unroll
             for (int k = 0; k < NS; ++k)
                 gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                if (LAYOUT == PAIRED) {
-                    const uint32_t wa = word(gv[0], q), wb = word(gv[1], q);
-                    GA[q] = f2(bf_lo(wa), bf_hi(wa));
-                    GB[q] = f2(bf_lo(wb), bf_hi(wb));
-                } else {
-                    const uint32_t w0 = word(gv[q >> 1], 2 * (q & 1));
-                    const uint32_t w1 = word(gv[q >> 1], 2 * (q & 1) + 1);
-                    GA[q] = f2(bf_lo(w0), bf_lo(w1));
-                    GB[q] = f2(bf_hi(w0), bf_hi(w1));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = word(gv[2 + k], i);
-                    GT[k][i] = f2(bf_lo(w), bf_hi(w));
-                }
+            unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
         }
+        RotCoef<NQ, NORM && !ROUND> kc;
+        make_coef(kc, C, Sn, GA, GB);
 
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            float2 A[NQ], B[NQ], TL[NT > 0 ? NT : 1][4];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                if (LAYOUT == PAIRED) {
-                    const uint32_t wa = word(raw[u][0], q), wb = word(raw[u][1], q);
-                    A[q] = f2(bf_lo(wa), bf_hi(wa));
-                    B[q] = f2(bf_lo(wb), bf_hi(wb));
-                } else {
-                    const uint32_t w0 = word(raw[u][q >> 1], 2 * (q & 1));
-                    const uint32_t w1 = word(raw[u][q >> 1], 2 * (q & 1) + 1);
-                    A[q] = f2(bf_lo(w0), bf_lo(w1));
-                    B[q] = f2(bf_hi(w0), bf_hi(w1));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = word(raw[u][2 + k], i);
-                    TL[k][i] = f2(bf_lo(w), bf_hi(w));
-                }
-
+            float2 A[NQ], B[NQ], TL[NTA][4];
+            unpack_row<LAYOUT, NS>(raw[u], A, B, TL);
+            float r = 1.f;
             if (NORM) {
-                float2 acc = f2(0.f, 0.f);
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    acc = __ffma2_rn(A[q], A[q], acc);
-                    acc = __ffma2_rn(B[q], B[q], acc);
-                }
-#pragma unroll
-                for (int k = 0; k < NT; ++k)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        acc = __ffma2_rn(TL[k][i], TL[k][i], acc);
-                float ss = acc.x + acc.y;
+                float ss = row_sumsq<LAYOUT, NS>(A, B, TL);
 #pragma unroll
                 for (int off = LPR / 2; off > 0; off >>= 1)
                     ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                const float r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
-                const float2 r2 = f2(r, r);
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    A[q] = __fmul2_rn(__fmul2_rn(A[q], r2), GA[q]);
-                    B[q] = __fmul2_rn(__fmul2_rn(B[q], r2), GB[q]);
-                    if (ROUND) {
-                        A[q] = round2_bf16(A[q]);
-                        B[q] = round2_bf16(B[q]);
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < NT; ++k)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        TL[k][i] = __fmul2_rn(__fmul2_rn(TL[k][i], r2), GT[k][i]);
+                r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
             }
-
-            // rotate: A' = A C - B S, B' = B C + A S (packed over two pairs)
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                const float2 bs = __fmul2_rn(B[q], Sn[q]);
-                const float2 bc = __fmul2_rn(B[q], C[q]);
-                const float2 a2 = __ffma2_rn(A[q], C[q], f2(-bs.x, -bs.y));
-                const float2 b2 = __ffma2_rn(A[q], Sn[q], bc);
-                A[q] = a2;
-                B[q] = b2;
-            }
-
+            norm_rotate<LAYOUT, NS, NORM, ROUND>(A, B, TL, r, kc, GA, GB, GT);
             uint4 outv[NS];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                if (LAYOUT == PAIRED) {
-                    set_word(outv[0], q, pack2(A[q].x, A[q].y));
-                    set_word(outv[1], q, pack2(B[q].x, B[q].y));
-                } else {
-                    set_word(outv[q >> 1], 2 * (q & 1), pack2(A[q].x, B[q].x));
-                    set_word(outv[q >> 1], 2 * (q & 1) + 1, pack2(A[q].y, B[q].y));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    set_word(outv[2 + k], i, pack2(TL[k][i].x, TL[k][i].y));
-
+            pack_row<LAYOUT, NS>(A, B, TL, outv);
             if (u < m.nh) {
 #pragma unroll
                 for (int k = 0; k < NS; ++k)

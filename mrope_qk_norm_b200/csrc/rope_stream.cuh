@@ -64,17 +64,57 @@ __device__ __forceinline__ uint4 *ring_at(uint4 *ring, int stage, int k)
     return ring + ((size_t)(stage * U * NS + k) * kThreads + threadIdx.x);
 }
 
+// Normalise, rotate and store the U rows of one work item from ring stage st.
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, bool ROUND>
+__device__ __forceinline__ void stream_rows(
+    const RopeParams &p, const Item &m, uint4 *ring, int st, const int (&vidx)[NS],
+    const float2 (&C)[RowShape<LAYOUT, NS>::NQ], const float2 (&Sn)[RowShape<LAYOUT, NS>::NQ],
+    const float2 (&GA)[RowShape<LAYOUT, NS>::NQ], const float2 (&GB)[RowShape<LAYOUT, NS>::NQ],
+    const float2 (&GT)[RowShape<LAYOUT, NS>::NTA][4])
+{
+    constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
+    constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
+    RotCoef<NQ, NORM && !ROUND> kc;
+    make_coef(kc, C, Sn, GA, GB);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        uint4 raw[NS];
+#pragma unroll
+        for (int k = 0; k < NS; ++k)
+            raw[k] = *ring_at<U, NS>(ring, st, u * NS + k);
+        float2 A[NQ], B[NQ], TL[NTA][4];
+        unpack_row<LAYOUT, NS>(raw, A, B, TL);
+        float r = 1.f;
+        if (NORM) {
+            float ss = row_sumsq<LAYOUT, NS>(A, B, TL);
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1)
+                ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
+        }
+        norm_rotate<LAYOUT, NS, NORM, ROUND>(A, B, TL, r, kc, GA, GB, GT);
+        uint4 outv[NS];
+        pack_row<LAYOUT, NS>(A, B, TL, outv);
+        if (u < m.nh) {
+#pragma unroll
+            for (int k = 0; k < NS; ++k)
+                if (vidx[k] >= 0)
+                    st_stream(m.dst + (int64_t)u * p.D + 8 * vidx[k], outv[k]);
+        }
+    }
+}
+
 template <int LAYOUT, int LPR, int NS, int U, bool NORM>
 __global__ void __launch_bounds__(kThreads)
 rope_stream_kernel(const __grid_constant__ RopeParams p)
 {
     pdl_wait();
     pdl_trigger();
-    constexpr int NQ = LAYOUT == PAIRED ? 4 : 2 * NS;
-    constexpr int NT = LAYOUT == PAIRED ? NS - 2 : 0;
+    constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
+    constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
     constexpr int G = kThreads / LPR;
     const int S = p.stages;
-    const bool ROUND = p.round_norm != 0;
+    const bool ROUND = p.round_norm != 0;  // uniform: both paths below are warp-uniform
 
     extern __shared__ float4 smem[];
     uint4 *ring = reinterpret_cast<uint4 *>(smem);
@@ -165,7 +205,7 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
                 Sn[q + 1] = f2(s4.z, s4.w);
             }
         }
-        float2 GA[NQ], GB[NQ], GT[NT > 0 ? NT : 1][4];
+        float2 GA[NQ], GB[NQ], GT[NTA][4];
         if (NORM) {
             const RopeStreamDev &Sd = m.s1 ? p.st[1] : p.st[0];
             const __nv_bfloat16 *gam = m.isk ? Sd.gk : Sd.gq;
@@ -173,124 +213,13 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
 #pragma unroll
             for (int k = 0; k < NS; ++k)
                 gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                if (LAYOUT == PAIRED) {
-                    const uint32_t wa = word(gv[0], q), wb = word(gv[1], q);
-                    GA[q] = f2(bf_lo(wa), bf_hi(wa));
-                    GB[q] = f2(bf_lo(wb), bf_hi(wb));
-                } else {
-                    const uint32_t w0 = word(gv[q >> 1], 2 * (q & 1));
-                    const uint32_t w1 = word(gv[q >> 1], 2 * (q & 1) + 1);
-                    GA[q] = f2(bf_lo(w0), bf_lo(w1));
-                    GB[q] = f2(bf_hi(w0), bf_hi(w1));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = word(gv[2 + k], i);
-                    GT[k][i] = f2(bf_lo(w), bf_hi(w));
-                }
+            unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
         }
 
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            uint4 raw[NS];
-#pragma unroll
-            for (int k = 0; k < NS; ++k)
-                raw[k] = *ring_at<U, NS>(ring, st, u * NS + k);
-            float2 A[NQ], B[NQ], TL[NT > 0 ? NT : 1][4];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                if (LAYOUT == PAIRED) {
-                    const uint32_t wa = word(raw[0], q), wb = word(raw[1], q);
-                    A[q] = f2(bf_lo(wa), bf_hi(wa));
-                    B[q] = f2(bf_lo(wb), bf_hi(wb));
-                } else {
-                    const uint32_t w0 = word(raw[q >> 1], 2 * (q & 1));
-                    const uint32_t w1 = word(raw[q >> 1], 2 * (q & 1) + 1);
-                    A[q] = f2(bf_lo(w0), bf_lo(w1));
-                    B[q] = f2(bf_hi(w0), bf_hi(w1));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = word(raw[2 + k], i);
-                    TL[k][i] = f2(bf_lo(w), bf_hi(w));
-                }
-
-            if (NORM) {
-                float2 acc = f2(0.f, 0.f);
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    acc = __ffma2_rn(A[q], A[q], acc);
-                    acc = __ffma2_rn(B[q], B[q], acc);
-                }
-#pragma unroll
-                for (int k = 0; k < NT; ++k)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        acc = __ffma2_rn(TL[k][i], TL[k][i], acc);
-                float ss = acc.x + acc.y;
-#pragma unroll
-                for (int off = LPR / 2; off > 0; off >>= 1)
-                    ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                const float r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
-                const float2 r2 = f2(r, r);
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    A[q] = __fmul2_rn(__fmul2_rn(A[q], r2), GA[q]);
-                    B[q] = __fmul2_rn(__fmul2_rn(B[q], r2), GB[q]);
-                    if (ROUND) {
-                        A[q] = round2_bf16(A[q]);
-                        B[q] = round2_bf16(B[q]);
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < NT; ++k)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        TL[k][i] = __fmul2_rn(__fmul2_rn(TL[k][i], r2), GT[k][i]);
-            }
-
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                const float2 bs = __fmul2_rn(B[q], Sn[q]);
-                const float2 bc = __fmul2_rn(B[q], C[q]);
-                const float2 a2 = __ffma2_rn(A[q], C[q], f2(-bs.x, -bs.y));
-                const float2 b2 = __ffma2_rn(A[q], Sn[q], bc);
-                A[q] = a2;
-                B[q] = b2;
-            }
-
-            uint4 outv[NS];
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-                if (LAYOUT == PAIRED) {
-                    set_word(outv[0], q, pack2(A[q].x, A[q].y));
-                    set_word(outv[1], q, pack2(B[q].x, B[q].y));
-                } else {
-                    set_word(outv[q >> 1], 2 * (q & 1), pack2(A[q].x, B[q].x));
-                    set_word(outv[q >> 1], 2 * (q & 1) + 1, pack2(A[q].y, B[q].y));
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < NT; ++k)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    set_word(outv[2 + k], i, pack2(TL[k][i].x, TL[k][i].y));
-
-            if (u < m.nh) {
-#pragma unroll
-                for (int k = 0; k < NS; ++k)
-                    if (vidx[k] >= 0)
-                        st_stream(m.dst + (int64_t)u * D + 8 * vidx[k], outv[k]);
-            }
-        }
+        if (ROUND)
+            stream_rows<LAYOUT, LPR, NS, U, NORM, true>(p, m, ring, st, vidx, C, Sn, GA, GB, GT);
+        else
+            stream_rows<LAYOUT, LPR, NS, U, NORM, false>(p, m, ring, st, vidx, C, Sn, GA, GB, GT);
     }
     cp_async_wait(0);  // nothing is left in flight (the trailing groups are empty)
     if (p.Hv > 0)

@@ -1,7 +1,7 @@
 // rope_tma.cu -- bulk-copy pipelined per-head RMSNorm + RoPE (sm_100a).
 //
-// Same arithmetic as the register kernel in rope_rows.cu (fused_qk_norm_rope,
-// vllm-omni #7600; mrope_apply, llama.cpp fork #286).  A memory-bound
+// Same arithmetic as the item kernel (the shared row math of rope_math.cuh;
+// fused_qk_norm_rope, vllm-omni #7600; mrope_apply, llama.cpp fork #286).  A memory-bound
 // kernel must keep tens of KB per SM in flight; here those bytes wait in a
 // shared-memory ring filled by the copy engine instead of in registers:
 //
@@ -31,7 +31,7 @@
 
 #include <climits>
 
-#include "qkr_internal.cuh"
+#include "rope_math.cuh"
 
 namespace qkr {
 
@@ -43,8 +43,6 @@ constexpr int kMaxConsumerThreads = 384;
 constexpr int kMaxThreads = 32 + kMaxConsumerThreads;
 constexpr int kStages = 4;
 constexpr long long kWaitBudgetCycles = 4000000000LL;  // ~2 s at 1.9 GHz
-
-enum Layout { PAIRED = 0, VECTOR = 1 };
 
 // ---------------------------------------------------------------- PTX -----
 
@@ -119,28 +117,6 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, volat
     return true;
 }
 
-// -------------------------------------------------------------- math ------
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
-__device__ __forceinline__ uint32_t word(const uint4 &v, int i)
-{
-    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
-__device__ __forceinline__ void set_word(uint4 &v, int i, uint32_t w)
-{
-    if (i == 0) v.x = w;
-    else if (i == 1) v.y = w;
-    else if (i == 2) v.z = w;
-    else v.w = w;
-}
-__device__ __forceinline__ float2 round2_bf16(float2 a)
-{
-    const uint32_t w = pack2(a.x, a.y);
-    return f2(bf_lo(w), bf_hi(w));
-}
-
 struct TileGeom {
     int64_t tok0;
     int ntok;
@@ -171,8 +147,8 @@ rope_tma_kernel(const __grid_constant__ RopeParams p, const __grid_constant__ Tm
 {
     pdl_wait();
     pdl_trigger();
-    constexpr int NQ = LAYOUT == PAIRED ? 4 : 2 * NS;
-    constexpr int NT = LAYOUT == PAIRED ? NS - 2 : 0;
+    constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
+    constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
 
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -304,7 +280,7 @@ rope_tma_kernel(const __grid_constant__ RopeParams p, const __grid_constant__ Tm
     __nv_bfloat16 *const obase = (isk ? p.k_out : p.q_out) + (int64_t)(have ? h : 0) * D;
     const int64_t ots = isk ? p.ko_ts : p.qo_ts;
 
-    float2 GA[NQ], GB[NQ], GT[NT > 0 ? NT : 1][4];
+    float2 GA[NQ], GB[NQ], GT[NTA][4];
     int gstream = -1;
     bool dead = false;  // a wait ran out: skip work but keep the barrier sequence
 
@@ -371,82 +347,20 @@ rope_tma_kernel(const __grid_constant__ RopeParams p, const __grid_constant__ Tm
 #pragma unroll
                     for (int k = 0; k < NS; ++k)
                         gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                    for (int q = 0; q < NQ; ++q) {
-                        if (LAYOUT == PAIRED) {
-                            const uint32_t wa = word(gv[0], q), wb = word(gv[1], q);
-                            GA[q] = f2(bf_lo(wa), bf_hi(wa));
-                            GB[q] = f2(bf_lo(wb), bf_hi(wb));
-                        } else {
-                            const uint32_t w0 = word(gv[q >> 1], 2 * (q & 1));
-                            const uint32_t w1 = word(gv[q >> 1], 2 * (q & 1) + 1);
-                            GA[q] = f2(bf_lo(w0), bf_lo(w1));
-                            GB[q] = f2(bf_hi(w0), bf_hi(w1));
-                        }
-                    }
-#pragma unroll
-                    for (int k = 0; k < NT; ++k)
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const uint32_t x = word(gv[2 + k], w);
-                            GT[k][w] = f2(bf_lo(x), bf_hi(x));
-                        }
+                    unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
                 }
 
-                float2 A[NQ], B[NQ], TL[NT > 0 ? NT : 1][4];
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    if (LAYOUT == PAIRED) {
-                        const uint32_t wa = word(raw[0], q), wb = word(raw[1], q);
-                        A[q] = f2(bf_lo(wa), bf_hi(wa));
-                        B[q] = f2(bf_lo(wb), bf_hi(wb));
-                    } else {
-                        const uint32_t w0 = word(raw[q >> 1], 2 * (q & 1));
-                        const uint32_t w1 = word(raw[q >> 1], 2 * (q & 1) + 1);
-                        A[q] = f2(bf_lo(w0), bf_lo(w1));
-                        B[q] = f2(bf_hi(w0), bf_hi(w1));
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < NT; ++k)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const uint32_t x = word(raw[2 + k], w);
-                        TL[k][w] = f2(bf_lo(x), bf_hi(x));
-                    }
+                float2 A[NQ], B[NQ], TL[NTA][4];
+                unpack_row<LAYOUT, NS>(raw, A, B, TL);
+                float r = 1.f;
                 if (NORM) {
-                    float2 acc = f2(0.f, 0.f);
-#pragma unroll
-                    for (int q = 0; q < NQ; ++q) {
-                        acc = __ffma2_rn(A[q], A[q], acc);
-                        acc = __ffma2_rn(B[q], B[q], acc);
-                    }
-#pragma unroll
-                    for (int k = 0; k < NT; ++k)
-#pragma unroll
-                        for (int w = 0; w < 4; ++w)
-                            acc = __ffma2_rn(TL[k][w], TL[k][w], acc);
-                    float ss = acc.x + acc.y;
+                    float ss = row_sumsq<LAYOUT, NS>(A, B, TL);
 #pragma unroll
                     for (int off = LPR / 2; off > 0; off >>= 1)
                         ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                    const float r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
-                    const float2 r2 = f2(r, r);
-#pragma unroll
-                    for (int q = 0; q < NQ; ++q) {
-                        A[q] = __fmul2_rn(__fmul2_rn(A[q], r2), GA[q]);
-                        B[q] = __fmul2_rn(__fmul2_rn(B[q], r2), GB[q]);
-                        if (ROUND) {
-                            A[q] = round2_bf16(A[q]);
-                            B[q] = round2_bf16(B[q]);
-                        }
-                    }
-#pragma unroll
-                    for (int k = 0; k < NT; ++k)
-#pragma unroll
-                        for (int w = 0; w < 4; ++w)
-                            TL[k][w] = __fmul2_rn(__fmul2_rn(TL[k][w], r2), GT[k][w]);
+                    r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
                 }
+                float2 C[NQ], Sn[NQ];
                 const float *cr = cosv + tt * cs_ld;
                 const float *sr = sinv + tt * cs_ld;
 #pragma unroll
@@ -456,34 +370,16 @@ rope_tma_kernel(const __grid_constant__ RopeParams p, const __grid_constant__ Tm
                                           : make_float4(1.f, 1.f, 1.f, 1.f);
                     const float4 s4 = okq ? *reinterpret_cast<const float4 *>(sr + qpair[q])
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float2 Cq[2] = {f2(c4.x, c4.y), f2(c4.z, c4.w)};
-                    const float2 Sq[2] = {f2(s4.x, s4.y), f2(s4.z, s4.w)};
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const float2 bs = __fmul2_rn(B[q + e], Sq[e]);
-                        const float2 bc = __fmul2_rn(B[q + e], Cq[e]);
-                        const float2 a2 = __ffma2_rn(A[q + e], Cq[e], f2(-bs.x, -bs.y));
-                        const float2 b2 = __ffma2_rn(A[q + e], Sq[e], bc);
-                        A[q + e] = a2;
-                        B[q + e] = b2;
-                    }
+                    C[q] = f2(c4.x, c4.y);
+                    C[q + 1] = f2(c4.z, c4.w);
+                    Sn[q] = f2(s4.x, s4.y);
+                    Sn[q + 1] = f2(s4.z, s4.w);
                 }
+                RotCoef<NQ, NORM && !ROUND> kc;
+                make_coef(kc, C, Sn, GA, GB);
+                norm_rotate<LAYOUT, NS, NORM, ROUND>(A, B, TL, r, kc, GA, GB, GT);
                 uint4 outv[NS];
-#pragma unroll
-                for (int q = 0; q < NQ; ++q) {
-                    if (LAYOUT == PAIRED) {
-                        set_word(outv[0], q, pack2(A[q].x, A[q].y));
-                        set_word(outv[1], q, pack2(B[q].x, B[q].y));
-                    } else {
-                        set_word(outv[q >> 1], 2 * (q & 1), pack2(A[q].x, B[q].x));
-                        set_word(outv[q >> 1], 2 * (q & 1) + 1, pack2(A[q].y, B[q].y));
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < NT; ++k)
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        set_word(outv[2 + k], w, pack2(TL[k][w].x, TL[k][w].y));
+                pack_row<LAYOUT, NS>(A, B, TL, outv);
                 __nv_bfloat16 *dst = obase + n * ots;
 #pragma unroll
                 for (int k = 0; k < NS; ++k)
