@@ -158,9 +158,13 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     ItemCursor icur, ccur;  // the pass being copied in, the pass being computed
     icur.start(grp, gpt);
     ccur = icur;
+    // With a two-pass ring the item a pass computes is the one the previous
+    // issue decoded: carry it instead of decoding it again.
+    Item carried;
     auto issue = [&](int pass) {
         if (pass < passes) {
             const Item m = decode_item<U>(p, tok0, icur, ntok, nbq);
+            carried = m;
             icur.advance(dq, dr, gpt);
             const int st = pass % S;
 #pragma unroll
@@ -181,10 +185,15 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     __syncthreads();
 
     for (int pass = 0; pass < passes; ++pass) {
+        Item m;
+        if (S == 2) {
+            m = carried;
+        } else {
+            m = decode_item<U>(p, tok0, ccur, ntok, nbq);
+            ccur.advance(dq, dr, gpt);
+        }
         issue(pass + S - 1);
         cp_async_wait(S - 1);
-        const Item m = decode_item<U>(p, tok0, ccur, ntok, nbq);
-        ccur.advance(dq, dr, gpt);
         const int st = pass % S;
 
         float2 C[NQ], Sn[NQ];
