@@ -302,8 +302,9 @@ qkr_status vit_mrope_setup(void *stream, const float *inv_t, const float *inv_h,
  * rms_norm_kernel): per row, s = bf16(x + residual) is written back to
  * residual, then out = s / sqrt(mean(s^2) + eps) * gamma (fp32 sum of
  * squares, one final bf16 rounding).  When rows are too few to fill the GPU
- * (a single decode row) each row is split across a thread-block cluster of
- * up to 16 CTAs whose partial sums meet in distributed shared memory.
+ * (decode: up to 32 rows) each row is split across a thread-block cluster of
+ * 8 (up to 8 rows) or 4 CTAs whose partial sums meet in distributed shared
+ * memory.
  *
  *   x                bf16 device [R, hidden], row stride x_stride.
  *   residual         bf16 device [R, hidden], in/out, row stride res_stride.
@@ -416,6 +417,14 @@ qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t token
  * (per-lane partial sums, then a shuffle tree), so results can differ in the
  * last bit between choices; each choice is deterministic. */
 qkr_status qkr_tune_rope_lanes(int32_t lanes);
+
+/* CTAs that share one row in rms_norm_residual / rms_norm_fp8, for tuning
+ * sweeps: 0 automatic (a cluster of 8 or 4 CTAs for up to 32 rows, else one
+ * CTA per row), else 1, 2, 4, 8 or 16 (a thread-block cluster when > 1).
+ * Process-wide.  The split sets the order of the fp32 sum of squares, so the
+ * normalised output can differ in the last bit between choices; the residual
+ * stream is bit-identical. */
+qkr_status qkr_tune_rms(int32_t cluster);
 
 /* Device status word of the library on the current device (0 = healthy).
  * Kernels that wait on shared-memory barriers give every wait a time budget;

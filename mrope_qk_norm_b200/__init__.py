@@ -29,7 +29,7 @@ KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange
 
 EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "rope_set_rows",
            "vit_mrope_setup", "rms_norm_residual", "rms_norm_fp8", "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
-           "qkr_vit_positions", "qkr_tune_rope", "qkr_tune_rope_lanes", "qkr_device_status",
+           "qkr_vit_positions", "qkr_tune_rope", "qkr_tune_rope_lanes", "qkr_tune_rms", "qkr_device_status",
            "qkr_launch_overlap")
 
 
@@ -94,6 +94,7 @@ def _load() -> ctypes.CDLL:
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
         "qkr_tune_rope": [I32, I32, I32, I32],
         "qkr_tune_rope_lanes": [I32],
+        "qkr_tune_rms": [I32],
         "qkr_launch_overlap": [I32],
         "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
     }
@@ -171,6 +172,11 @@ def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 
 def tune_rope_lanes(lanes: int = 0) -> None:
     """Lanes per head row of the GPT-J layout (0 = automatic), for tuning."""
     _check(_lib.qkr_tune_rope_lanes(lanes))
+
+
+def tune_rms(cluster: int = 0) -> None:
+    """CTAs per row of the RMSNorm kernels (0 = automatic), for tuning."""
+    _check(_lib.qkr_tune_rms(cluster))
 
 
 def launch_overlap(enable: bool) -> None:

@@ -445,6 +445,16 @@ qkr_status qkr_launch_overlap(int32_t enable)
     return QKR_OK;
 }
 
+qkr_status qkr_tune_rms(int32_t cluster)
+{
+    if (cluster != 0 && cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8 &&
+        cluster != 16)
+        return fail(QKR_ERR_INVALID_ARG, "cluster must be 0 or a power of two up to 16");
+    qkr::set_rms_cluster_override(cluster);
+    g_error.clear();
+    return QKR_OK;
+}
+
 qkr_status qkr_tune_rope_lanes(int32_t lanes)
 {
     if (lanes != 0 && lanes != 1 && lanes != 2 && lanes != 4 && lanes != 8 && lanes != 16)

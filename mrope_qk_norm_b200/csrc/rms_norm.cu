@@ -9,8 +9,8 @@
 // registers, so the row crosses HBM exactly once (read x and residual, write
 // residual and out).  The occupancy problem of vllm.cpp #185 (one workgroup
 // per row leaves the GPU idle when a decode step has one row) is solved with
-// a thread-block cluster: when rows are too few to fill the 148 SMs, each row
-// is split across a cluster of up to 16 CTAs, every CTA reduces its slice,
+// a thread-block cluster: when rows are few (up to 32), each row is split
+// across a cluster of 4 or 8 CTAs, every CTA reduces its slice,
 // the partial sums are exchanged through distributed shared memory (read by
 // every CTA in rank order, so all CTAs get the same bit-identical total), and
 // each CTA normalises its slice.  No global scratch, no atomics, no spin-wait
@@ -199,14 +199,7 @@ Fn cluster_fn(int vpt)
     }
 }
 
-int sm_count()
-{
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-        return 148;
-    return n;
-}
+int g_force_cluster = 0;  // tuning override of CTAs per row (0: automatic)
 
 // Smallest power-of-two vectors-per-thread keeping the block at or under
 // `target` threads (and never above 1024).
@@ -223,16 +216,23 @@ void shape(int vectors, int target, int &vpt, int &threads)
 
 }  // namespace
 
+void set_rms_cluster_override(int cluster) { g_force_cluster = cluster; }
+
 cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, LaunchRecord *rec)
 {
     const bool fp8 = p.out8 != nullptr;
     const int nvec = p.hidden >> 3;
-    const int target_ctas = 2 * sm_count();
-    int cs = 1;
-    if (p.R < target_ctas) {
-        while (cs < 16 && p.R * cs < target_ctas && nvec / (2 * cs) >= 32)
-            cs <<= 1;
-    }
+    // CTAs per row.  A sweep on B200 (hidden 5120 / 8192, R = 1 .. 128) put the
+    // best split at 8 CTAs for up to 8 rows, 4 for up to 32 and one CTA per row
+    // beyond: a cluster launch and its DSMEM exchange cost more than the extra
+    // SMs save once a few rows are in flight (R = 32: 2.61 us at 4 per row vs
+    // 3.54 us at 16; R = 128: 3.98 us at 1 vs 4.81 us at 4).  A slice keeps at
+    // least 32 vectors per CTA.
+    int cs = p.R <= 8 ? 8 : (p.R <= 32 ? 4 : 1);
+    while (cs > 1 && nvec / cs < 32)
+        cs >>= 1;
+    if (g_force_cluster > 0 && nvec / g_force_cluster >= 1)
+        cs = g_force_cluster;
     int vpt, threads;
     const int per = (nvec + cs - 1) / cs;
     shape(per, 256, vpt, threads);
