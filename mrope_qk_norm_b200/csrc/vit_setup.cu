@@ -45,6 +45,22 @@ __device__ __forceinline__ void token_position(const int32_t *cu, const int32_t 
     const int h = grids[3 * g + 1];
     const int w = grids[3 * g + 2];
     const int64_t frame = max((int64_t)h * w, (int64_t)1);
+    if (frame <= 0xffffffffLL && local >= 0 && local <= 0xffffffffLL && m > 0) {
+        // the usual case, in 32-bit unsigned arithmetic (a 64-bit division is
+        // several times longer, and this chain is the CTA's critical path)
+        const uint32_t l32 = (uint32_t)local, f32 = (uint32_t)frame, mm = (uint32_t)(m * m);
+        const uint32_t t32 = l32 / f32;
+        const uint32_t in_frame = l32 - t32 * f32;
+        const uint32_t block = in_frame / mm;
+        const uint32_t patch = in_frame - block * mm;
+        const uint32_t bpr = (uint32_t)max(w / m, 1);
+        const uint32_t brow = block / bpr;
+        const uint32_t bcol = block - brow * bpr;
+        tp = (int)t32;
+        hp = (int)(brow * (uint32_t)m + patch / (uint32_t)m);
+        wp = (int)(bcol * (uint32_t)m + patch % (uint32_t)m);
+        return;
+    }
     tp = (int)(local / frame);
     const int64_t in_frame = local - (int64_t)tp * frame;
     const int mm = m * m;
