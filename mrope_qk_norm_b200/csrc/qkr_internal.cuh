@@ -190,7 +190,7 @@ struct LaunchRecord {
 };
 
 // Launch-shape override of the rope kernels (0: automatic); pipeline: 0 auto,
-// 1 register kernel only, 2 bulk-copy pipelined kernel only.
+// 1 item kernel only, 2 bulk-copy pipelined kernel only, 3 streaming kernel only.
 void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta,
                              int stages);
 // Lanes per head row of the GPT-J (VECTOR) layout, for tuning (0: automatic).

@@ -454,7 +454,8 @@ int sm_count()
 }  // namespace
 
 // Returns cudaErrorNotSupported when the call is outside what the pipelined
-// kernel serves (the caller then uses the register kernel).
+// kernel serves (joint V, scatter): it is reached only when a caller forces it
+// through qkr_tune_rope, and such a call then fails with QKR_ERR_CUDA.
 cudaError_t launch_rope_tma(const RopeParams &p_in, int layout_paired, int lpr, int ns,
                             int tokens_per_tile, cudaStream_t stream, LaunchRecord *rec)
 {
