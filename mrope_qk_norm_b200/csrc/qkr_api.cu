@@ -323,6 +323,10 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     }
     if (T > ((int64_t)1 << 40))
         return fail(QKR_ERR_INVALID_ARG, "token count too large");
+    if (T > INT32_MAX)
+        return fail(QKR_ERR_UNSUPPORTED,
+                    "%lld tokens in one launch: the kernels take at most 2^31 - 1; split the "
+                    "call into chunks with a token offset", (long long)T);
     const int64_t k_rows_out = k_only ? k_out_rows : T;
     if (!view_fits(T, qo_ts, 1, 0, Hq * D) || !view_fits(k_rows_out, ko_ts, 1, 0, Hk * D))
         return fail(QKR_ERR_INVALID_ARG, "output view exceeds the address range");

@@ -248,3 +248,17 @@ def test_rms_norm_fp8_refusals(qkr):
     assert call(hidden=60, xs=60, rs=60, os=60) == U
     assert call(R=0) == qkr.QKR_OK
     assert qkr.last_launch()["launches"] == 0
+
+
+def test_too_many_tokens_is_refused_not_launched(qkr):
+    L = qkr.lib()
+    T = 1 << 31  # one past what a launch takes
+    d = qkr.StreamDesc(q=FAKE, k=FAKE + (1 << 40), q_offset=0, k_offset=0, q_tok_stride=64,
+                       q_head_stride=64, k_tok_stride=64, k_head_stride=64, n_tokens=T,
+                       gamma_q=FAKE + (2 << 40), gamma_k=FAKE + (2 << 40))
+    a = qkr.AngleDesc(kind=qkr.ANGLE_TABLE, section_mode=0, cos=FAKE + (3 << 40),
+                      sin=FAKE + (4 << 40), table_rows=T, ld=32, plane_stride=32 * T)
+    arr = (qkr.StreamDesc * 1)(d)
+    st = L.fused_qk_norm_rope(None, arr, 1, FAKE + (5 << 40), FAKE + (6 << 40), 64, 64, 1, 1, 64,
+                              64, 0, 1e-6, ctypes.byref(a), 0)
+    assert st == qkr.QKR_ERR_UNSUPPORTED and "2^31" in _err(qkr)
