@@ -138,8 +138,8 @@ typedef struct qkr_stream_desc {
  *   positions      device int32 [rows, pos_row_stride]; rows = 1 (NONE),
  *                  3 (CONTIGUOUS / INTERLEAVED*), 4 (IMROPE).
  *   pos_row_stride elements between rows = tokens the buffer covers
- *                  (llama.cpp fork #286: a chunk keeps the whole positions
- *                  buffer and is told where its tokens start).
+ *                  (llama.cpp fork #286: a launch over part of the tokens
+ *                  indexes the full-length rows from token_offset on).
  *   inv_freq       device fp32 [P], P = rot_dim / 2.
  *   cos, sin       device fp32 tables; table_rows tokens per plane, ld >= P
  *                  elements between token rows, plane_stride elements
@@ -213,9 +213,9 @@ qkr_status fused_qkv_norm_rope(void *stream, const qkr_stream_desc *streams, int
 
 /*
  * mrope_apply -- multi-section RoPE (llama.cpp fork #286, "The change":
- * each rotated pair reads the position section its index selects; a launch
- * over a token chunk keeps the whole positions buffer and is told where its
- * tokens start).  Rotates Q [T, Hq, D] and K [T, Hkv, D] (heads dense, token
+ * the section a pair falls in picks the position row its angle comes from;
+ * a launch over part of the tokens indexes the full-length position rows from
+ * its first token).  Rotates Q [T, Hq, D] and K [T, Hkv, D] (heads dense, token
  * strides given) with angles from positions + inv_freq, pair j reading row
  * section(j) at column token_offset + t.  If gamma_q and gamma_k are both
  * non-NULL each head is RMS-normalised first (as fused_qk_norm_rope); both

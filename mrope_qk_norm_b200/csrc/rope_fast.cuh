@@ -2,9 +2,9 @@
 //
 // One kernel template serves fused_qk_norm_rope (vllm-omni #7600: per-stream
 // per-head RMSNorm of Q and K, text-first concatenation and RoPE in one
-// launch) and mrope_apply (llama.cpp fork #286: each rotated pair reads the
-// position row its section selects; a chunk reads the whole positions buffer
-// from a token offset).  Its instantiations are split over several
+// launch) and mrope_apply (llama.cpp fork #286: the section a pair falls in
+// picks the position row its angle comes from; a launch over part of the
+// tokens indexes the full-length position rows from its first token).  Its instantiations are split over several
 // translation units (rope_fast_*.cu) so they compile in parallel; each unit
 // exports one picker.
 //

@@ -2,8 +2,8 @@
 
 Tokens are independent, so a batch splits into contiguous token ranges, one
 per rank, with no exchange step.  A shard is exactly a chunked launch
-(llama.cpp fork #286, "The change": a launch over a token chunk keeps the
-whole positions buffer and is told where its tokens start): rank r processes
+(llama.cpp fork #286, "The change": a launch over part of the tokens indexes
+the full-length position rows from its first token): rank r processes
 tokens [t0, t1) of its inputs and passes ``token_offset = t0`` so angles are
 read for the right tokens.
 """

@@ -2,8 +2,8 @@
 
 Full interleaved configuration: T=8192, Hq=16, Hkv=8, D=128, sections
 (24, 20, 20), three independent position rows in [0, 8192), theta=5e6, NeoX,
-also as two chunked launches split at token 2457 with a token offset into the
-whole positions buffer.  Section maps and chunking are checked bit-exactly.
+also as two chunked launches split at token 2457, each with a token offset into the
+full-length position rows.  Section maps and chunking are checked bit-exactly.
 """
 import numpy as np
 import pytest

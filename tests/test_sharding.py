@@ -1,7 +1,7 @@
 """Token-range sharding across ranks (gloo, world size 2, CPU).
 
 Each rank computes its shard with the CPU oracle using the shard's token
-offset into the whole positions buffer; rank 0 gathers the shards and checks
+offset into the full-length position rows; rank 0 gathers the shards and checks
 that they equal the unsharded result bit for bit.  This exercises the host
 logic of the multi-GPU path (token ranges, offsets, gathering) without a GPU.
 """
