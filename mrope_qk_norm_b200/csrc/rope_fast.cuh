@@ -4,9 +4,9 @@
 // per-head RMSNorm of Q and K, text-first concatenation and RoPE in one
 // launch) and mrope_apply (llama.cpp fork #286: the section a pair falls in
 // picks the position row its angle comes from; a launch over part of the
-// tokens indexes the full-length position rows from its first token).  Its instantiations are split over several
-// translation units (rope_fast_*.cu) so they compile in parallel; each unit
-// exports one picker.
+// tokens indexes the full-length position rows from its first token).  Its
+// instantiations are split over several translation units (rope_fast_*.cu) so
+// they compile in parallel; each unit exports one picker.
 //
 // B200 mapping.  The op moves ~4 bytes per element and does a handful of
 // flops on it, so it is HBM-bound only if the instruction stream stays lean:
