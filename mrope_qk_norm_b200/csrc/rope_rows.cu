@@ -238,11 +238,12 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
                                          (int)(ring + angles_max));
     if (e != cudaSuccess)
         return e;
-    // Token split: 8 tokens per CTA once that still gives four waves of
-    // resident CTAs, else 4.  On interleaved mRoPE (8192 x (16+8) heads,
-    // whole and chunked at 2457) this was within 3% of the best fixed split
-    // in each case; a single wave of larger ranges was 3-15% slower (each
-    // CTA's staging prologue is exposed once per range).
+    // Token split: 8 tokens per CTA once that still fills a wave of resident
+    // CTAs, else 4.  On interleaved mRoPE (8192 x (16+8) heads) launches of
+    // 8192 and 5735 tokens were fastest at 8 and one of 2457 at 4 (8.5 us
+    // against 9.3 us at 8, whose grid is half a wave); 16 tokens per CTA
+    // was 8-13% slower on all three (each CTA's staging prologue is exposed
+    // once per range, over fewer CTAs).
     int64_t grid;
     int tt = g_force_tt;
     if (tt <= 0) {
@@ -250,7 +251,14 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
         e = resident_slots(fn, ring + (size_t)8 * cs_ld * 2 * sizeof(float), &slots);
         if (e != cudaSuccess)
             return e;
-        tt = p.T >= 4 * (int64_t)slots ? 8 : 4;
+        tt = p.T >= 8 * (int64_t)slots ? 8 : 4;
+        // Few heads per token (K-only scatter into a cache: 8 heads, 4
+        // items per token) would leave one item per lane group at 8
+        // tokens, so nothing overlaps the ring's first wait; 16 tokens
+        // measured 5% faster on 8192 x 8 heads of K.
+        const int items_per_token = (p.Hq + u - 1) / u + (p.Hk + u - 1) / u;
+        if (tt == 8 && 8 * items_per_token < 2 * (kThreads / lpr))
+            tt = 16;
     }
     if (tt > kStreamTokens)
         tt = kStreamTokens;
@@ -275,6 +283,25 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
         rec->launches = 1;
     }
     return e;
+}
+
+// Resident CTAs of the automatic streaming shape (U = 2, S = 2, 8 tokens of
+// staged angles) for this call's layout.
+cudaError_t stream_slots(const RopeParams &p, int layout, int lpr, int ns, int *slots)
+{
+    const int pw = layout == VECTOR ? p.D / 2 : p.P;
+    const int cs_ld = (pw + 3) & ~3;
+    KernelFn fn = layout == PAIRED ? pick_stream_paired(lpr, ns, 2, p.norm != 0)
+                                   : pick_stream_vector(lpr, ns, 2, p.norm != 0);
+    if (!fn)
+        return cudaErrorInvalidConfiguration;
+    const size_t ring = (size_t)2 * 2 * ns * kThreads * 16;
+    const size_t angles_max = (size_t)kStreamTokens * cs_ld * 2 * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(ring + angles_max));
+    if (e != cudaSuccess)
+        return e;
+    return resident_slots(fn, ring + (size_t)8 * cs_ld * 2 * sizeof(float), slots);
 }
 
 int pow2_ceil(int v)
@@ -334,7 +361,21 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     // faster than the item kernel's per-4-token staging on interleaved mRoPE
     // (8192 x (16+8) heads); angles from a table: the item kernel with direct
     // 16-byte table reads measured ~12% faster than the streaming kernel.
-    const bool stream_auto = g_force_pipe == 0 && p.angle_kind == QKR_ANGLE_POSITIONS;
+    // Below a wave of streaming CTAs at 4 tokens each the item kernel with
+    // 4-token staging is the faster one: 1024 tokens of interleaved mRoPE
+    // (16+8 heads) took 3.7 us against 4.3 us, 16 tokens of 4+4 heads 2.5
+    // against 2.8.  Above it the gain is small (2457 tokens: 8.3 against
+    // 8.5 us) and is lost when a streaming launch follows directly: two
+    // chunks of 2457 and 5735 tokens took 24.2 us with the first on the item
+    // kernel against 23.7 us with both streaming.
+    bool stream_auto = g_force_pipe == 0 && p.angle_kind == QKR_ANGLE_POSITIONS;
+    if (stream_auto && layout != EXCHANGE && g_force_tt <= 0) {
+        int slots = 0;
+        const cudaError_t e = stream_slots(p, layout, lpr, ns, &slots);
+        if (e != cudaSuccess)
+            return e;
+        stream_auto = p.T >= 4 * (int64_t)slots;
+    }
     if (layout != EXCHANGE && (g_force_pipe == 3 || stream_auto))
         return launch_rope_stream(p, layout, lpr, ns, stream, rec);
     // staged (cos, sin) columns: GPT-J stages every pair of the head so pairs

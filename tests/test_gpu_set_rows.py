@@ -141,3 +141,20 @@ def test_out_of_range_row_is_skipped_and_reported():
     named = np.zeros(R, dtype=bool)
     named[idx[good]] = True
     assert cache.untouched()[~named].all()
+
+
+def test_scatter_full_size():
+    """The measured size: 8192 tokens x 8 K heads into a 16384-row cache, in
+    the launch shape the launcher picks for it (16 tokens per CTA)."""
+    w = _case(W.SECTIONS_INTERLEAVED, T=8192, seed=521)
+    R = 16384
+    idx = np.random.default_rng(21).permutation(R)[:8192]
+    cache = _scatter(w, idx, R)
+    rec = qkr.last_launch()
+    assert rec["pipelined"] == 2 and rec["tokens_per_cta"] == 16, rec
+    rid = torch.as_tensor(idx, dtype=torch.int64, device="cuda")
+    assert torch.equal(_bits(cache.tensor[rid]), _bits(_mrope_k(w))), "scatter != mrope_apply"
+    assert cache.untouched()[np.setdiff1d(np.arange(R), idx)].all()
+    _, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle,
+                                norm=False)
+    assert_bf16_close(cache.tensor[rid], rk, "full-size scatter")
