@@ -174,6 +174,40 @@ int g_force_tt = 0;    // tuning override of tokens per CTA (0: automatic)
 int g_force_s = 0;     // tuning override of the streaming ring depth (0: automatic)
 int g_force_lpr = 0;   // tuning override of lanes per row, GPT-J layout (0: automatic)
 
+// Opts `fn` in to `bytes` of dynamic shared memory on the current device.
+// The largest size already granted per (device, kernel) is cached, so a
+// launch after the first costs no driver call.
+cudaError_t allow_smem(KernelFn fn, size_t bytes)
+{
+    struct Entry {
+        int dev;
+        KernelFn fn;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> granted;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry *hit = nullptr;
+    for (Entry &g : granted)
+        if (g.dev == dev && g.fn == fn) {
+            if (g.bytes >= bytes)
+                return cudaSuccess;
+            hit = &g;
+        }
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess)
+        return e;
+    if (hit)
+        hit->bytes = bytes;
+    else
+        granted.push_back({dev, fn, bytes});
+    return cudaSuccess;
+}
+
 // CTAs of `fn` (256 threads, `smem` bytes of dynamic shared memory) resident
 // on the whole current device at once.  Cached per (device, kernel, smem).
 cudaError_t resident_slots(KernelFn fn, size_t smem, int *slots)
@@ -234,8 +268,7 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
         return cudaErrorInvalidConfiguration;
     const size_t ring = (size_t)S * u * ns * kThreads * 16;
     const size_t angles_max = (size_t)kStreamTokens * cs_ld * 2 * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(ring + angles_max));
+    cudaError_t e = allow_smem(fn, ring + angles_max);
     if (e != cudaSuccess)
         return e;
     // Token split: 8 tokens per CTA once that still fills a wave of resident
@@ -297,8 +330,7 @@ cudaError_t stream_slots(const RopeParams &p, int layout, int lpr, int ns, int *
         return cudaErrorInvalidConfiguration;
     const size_t ring = (size_t)2 * 2 * ns * kThreads * 16;
     const size_t angles_max = (size_t)kStreamTokens * cs_ld * 2 * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(ring + angles_max));
+    const cudaError_t e = allow_smem(fn, ring + angles_max);
     if (e != cudaSuccess)
         return e;
     return resident_slots(fn, ring + (size_t)8 * cs_ld * 2 * sizeof(float), slots);
@@ -444,8 +476,7 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
         smem += (size_t)groups * p.D * sizeof(float);
     smem = (smem + 15) & ~(size_t)15;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        const cudaError_t e = allow_smem(fn, smem);
         if (e != cudaSuccess)
             return e;
     }
