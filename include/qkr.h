@@ -404,7 +404,8 @@ qkr_status qkr_launch_overlap(int32_t enable);
  * streaming kernel takes 1, 2 or 4), tokens per CTA or per pipeline tile
  * (1..64; kernels that stage angles cap it by their shared memory) and ring
  * depth of the streaming kernel (2..4); 0 keeps the automatic choice.
- * Process-wide.  Every shape computes bit-identical results: a row's
+ * Process-wide; a launch racing a change on another thread takes the old or
+ * the new value of each knob.  Every shape computes bit-identical results: a row's
  * arithmetic does not depend on it.  Returns QKR_ERR_INVALID_ARG out of
  * range. */
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,

@@ -19,6 +19,7 @@
 #include <cooperative_groups.h>
 #include <cuda_fp8.h>
 
+#include <atomic>
 #include <climits>
 
 #include "qkr_internal.cuh"
@@ -199,7 +200,7 @@ Fn cluster_fn(int vpt)
     }
 }
 
-int g_force_cluster = 0;  // tuning override of CTAs per row (0: automatic)
+std::atomic<int> g_force_cluster{0};  // tuning override of CTAs per row (0: automatic)
 
 // Smallest power-of-two vectors-per-thread keeping the block at or under
 // `target` threads (and never above 1024).

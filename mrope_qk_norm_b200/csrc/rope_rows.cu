@@ -6,6 +6,7 @@
 // rot_dim % 16 != 0 (EXCHANGE layout) is served by a plainer kernel here that
 // passes the normalised row through shared memory to reach partners.
 
+#include <atomic>
 #include <climits>
 #include <mutex>
 #include <vector>
@@ -168,11 +169,13 @@ KernelFn pick_exchange(int lpr, int ns)
 #undef QKR_EXCHANGE_CASE
 }
 
-int g_force_pipe = 0;  // 0 automatic, 1 item kernel, 2 bulk-copy kernel, 3 streaming kernel
-int g_force_u = 0;     // tuning override of heads per item (0: automatic)
-int g_force_tt = 0;    // tuning override of tokens per CTA (0: automatic)
-int g_force_s = 0;     // tuning override of the streaming ring depth (0: automatic)
-int g_force_lpr = 0;   // tuning override of lanes per row, GPT-J layout (0: automatic)
+// Process-wide tuning overrides (atomics: a knob set from one thread while
+// another launches is a race on the launch shape only, never on memory).
+std::atomic<int> g_force_pipe{0};  // 0 automatic, 1 item, 2 bulk-copy, 3 streaming kernel
+std::atomic<int> g_force_u{0};     // heads per item (0: automatic)
+std::atomic<int> g_force_tt{0};    // tokens per CTA (0: automatic)
+std::atomic<int> g_force_s{0};     // streaming ring depth (0: automatic)
+std::atomic<int> g_force_lpr{0};   // lanes per row, GPT-J layout (0: automatic)
 
 // Opts `fn` in to `bytes` of dynamic shared memory on the current device.
 // The largest size already granted per (device, kernel) is cached, so a
@@ -254,10 +257,11 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
 {
     // U = 2 heads per item with a two-pass ring was the best streaming shape
     // in the sweeps (deeper rings and U = 4 cost resident CTAs).
-    int u = g_force_u > 0 ? g_force_u : 2;
+    const int fu = g_force_u, fs = g_force_s;
+    int u = fu > 0 ? fu : 2;
     if (u == 3)
         u = 2;
-    const int S = g_force_s > 0 ? g_force_s : 2;
+    const int S = fs > 0 ? fs : 2;
     p.stages = S;
     p.pw = layout == VECTOR ? p.D / 2 : p.P;
     const int cs_ld = (p.pw + 3) & ~3;
@@ -454,7 +458,8 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
 
     int64_t grid;
     if (g_force_tt > 0) {
-        const int tt = g_force_tt < max_tt_smem ? g_force_tt : max_tt_smem;
+        const int ftt = g_force_tt;
+        const int tt = ftt < max_tt_smem ? ftt : max_tt_smem;
         grid = (p.T + tt - 1) / tt;
     } else if (direct) {
         int slots = 0;
