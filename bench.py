@@ -79,7 +79,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device: torch.device, period_s: float = 0.005):
+    def __init__(self, device: torch.device, period_s: float = 0.001):
         self.samples = []
         self.ok = False
         self.period = period_s
@@ -119,16 +119,24 @@ class ClockSampler:
             self._t.join()
 
     def summary(self, t0: float, t1: float) -> dict:
+        """Median SM clock and the throttle reasons seen by the samples taken
+        inside [t0, t1] (host clock); says so when there are none."""
         if not self.ok:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
-        win = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"],
+                    "samples": 0}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": ["no clock sample inside the timed window"], "samples": 0,
+                    "window_ms": round(1e3 * (t1 - t0), 3)}
         mhz = [s[1] for s in win]
         mask = 0
         for s in win:
             mask |= s[2]
         reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
-        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(win)}
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(win),
+                "window_ms": round(1e3 * (t1 - t0), 3), "period_ms": 1e3 * self.period}
 
 
 # ------------------------------------------------------- headline (fused) --
@@ -165,12 +173,14 @@ class FusedSet:
                                     self.w.eps, self.angle, 0, stream)
 
 
-def time_launches(fns, steps, warmup, stream):
+def time_launches(fns, steps, warmup, stream, reps=5):
     """Run fns[i % len] `steps` times; returns (total_ms, per-launch ms list).
 
-    The `steps` launches are captured into one CUDA graph and replayed once,
-    so host-side call overhead (a few us per ctypes call) does not hide the
-    device time of small kernels; per-launch time is the graph time / steps.
+    The `steps` launches are captured into one CUDA graph, so host-side call
+    overhead (a few us per ctypes call) does not hide the device time of
+    small kernels.  After an upload replay, an untimed replay runs ahead of
+    `reps` timed back-to-back replays (each between its own CUDA events);
+    total_ms is the median replay, and per-launch time is that / steps.
     """
     with torch.cuda.stream(stream):
         for i in range(max(warmup, len(fns))):
@@ -183,13 +193,15 @@ def time_launches(fns, steps, warmup, stream):
     with torch.cuda.stream(stream):
         g.replay()  # untimed replay: first replay uploads the graph
     torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
     with torch.cuda.stream(stream):
-        start.record(stream)
-        g.replay()
-        end.record(stream)
+        g.replay()  # lead replay: the GPU is busy when the first event is recorded
+        evs[0].record(stream)
+        for i in range(reps):
+            g.replay()
+            evs[i + 1].record(stream)
     torch.cuda.synchronize()
-    total = start.elapsed_time(end)
+    total = statistics.median([evs[i].elapsed_time(evs[i + 1]) for i in range(reps)])
     del g
     return total, [total / steps] * steps
 
@@ -543,6 +555,8 @@ def main():
     ap.add_argument("--no-rows", action="store_true", help="skip the per-kernel rows")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--timed-ms", type=float, default=200.0,
+                    help="length of the timed region: back-to-back replays of the K-step graph")
     ap.add_argument("--row-steps", type=int, default=200)
     ap.add_argument("--row-warmup", type=int, default=20)
     ap.add_argument("--no-rms-sweep", action="store_true",
@@ -583,7 +597,7 @@ def main():
 
     sampler = ClockSampler(dev)
     sampler.start()
-    # warm-up (untimed), then K steps captured in one graph and replayed once
+    # warm-up (untimed), then K steps captured in one graph
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             fns[i % n_sets]()
@@ -592,25 +606,47 @@ def main():
     with torch.cuda.graph(graph, stream=stream):
         for i in range(args.steps):
             fns[i % n_sets]()
+    # untimed replays: the first uploads the graph, the second sizes the timed region
     with torch.cuda.stream(stream):
-        graph.replay()  # untimed: uploads the graph
+        graph.replay()
     torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        p0.record(stream)
+        graph.replay()
+        p1.record(stream)
+    torch.cuda.synchronize()
+    probe_ms = max(p0.elapsed_time(p1), 1e-3)
+    # Timed region: R back-to-back replays of the K-step graph (R so that the
+    # region lasts about --timed-ms), each bracketed by its own events; an
+    # untimed replay enqueued just before the first event keeps the GPU busy,
+    # so host submission never falls inside a timed replay.  Reported: the
+    # median replay, i.e. the time of exactly K steps.
+    reps = max(1, min(10000, int(np.ceil(args.timed_ms / probe_ms))))
+    if dist:
+        import torch.distributed as dist_mod
+        r_t = torch.tensor([reps], dtype=torch.int64, device=dev)
+        dist_mod.all_reduce(r_t, op=dist_mod.ReduceOp.MAX)
+        reps = int(r_t.item())
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        ev0.record(stream)
-        graph.replay()
-        ev1.record(stream)
+        graph.replay()  # lead replay (untimed)
+        evs[0].record(stream)
+        for i in range(reps):
+            graph.replay()
+            evs[i + 1].record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.perf_counter()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.stop()
-    total_ms = ev0.elapsed_time(ev1)
+    rep_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
+    total_ms = statistics.median(rep_ms)
     per = [total_ms / args.steps]
     del graph
     info = qkr.last_launch()
@@ -726,6 +762,10 @@ def main():
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": tokens,
+                   "timing": "median of %d back-to-back replays of a %d-step graph (each "
+                             "replay between its own CUDA events; an untimed replay runs "
+                             "ahead of the first); replay spread %.4f-%.4f ms"
+                             % (reps, args.steps, min(rep_ms), max(rep_ms)),
                    "parallelism": "dp%d (independent batches, no collective)" % world,
                    "l2": "%d rotating input/output sets of %.1f MB (%.0f MB > 2x126 MB L2)"
                          % (n_sets, nbytes / 1e6, n_sets * nbytes / 1e6)},
@@ -745,7 +785,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "path": "pinned host -> H2D stream | fused_qk_norm_rope stream | D2H stream "
                         "(two device buffer sets, consecutive steps overlap)"},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * reps,
         "clocks": clocks,
         "rows": rows,
         "rms_sweep": sweep,

@@ -223,7 +223,11 @@ qkr_status fused_qkv_norm_rope(void *stream, const qkr_stream_desc *streams, int
  *
  *   q, k             bf16 device inputs; q_out, k_out bf16 device outputs.
  *                    In-place is allowed: q_out == q with the same token
- *                    stride (likewise k); any other overlap is refused.
+ *                    stride (likewise k).  Views that share no element are
+ *                    accepted even where their byte ranges interleave (Q and
+ *                    K as column windows of one packed [T, 3, H, D] buffer
+ *                    with one token stride, rotated in place); any other
+ *                    overlap is refused.
  *   positions        device int32 [n_rows, T_total]; n_rows must match the
  *                    section mode (1 NONE, 3 sectioned, 4 IMROPE).
  *   token_offset     first token of this launch within positions;
@@ -360,7 +364,8 @@ enum {
     QKR_KERNEL_RMS_ROWS = 5,       /* one CTA per row */
     QKR_KERNEL_RMS_CLUSTER = 6,    /* one cluster per row */
     QKR_KERNEL_SECTION_MAP = 7,
-    QKR_KERNEL_VIT_POSITIONS = 8
+    QKR_KERNEL_VIT_POSITIONS = 8,
+    QKR_KERNEL_NULL = 9            /* qkr_null_launch */
 };
 typedef struct qkr_launch_info {
     int32_t kernel;          /* QKR_KERNEL_* */
@@ -368,11 +373,10 @@ typedef struct qkr_launch_info {
     int32_t slots;           /* rope: 16-byte vectors per lane per row; rms: per thread */
     int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
     int32_t heads_per_item;  /* rope: head rows of one token a lane group loads
-                                together (pipelined kernel: head slots per CTA) */
+                                together */
     int32_t pipelined;       /* rope: 0 rows loaded straight into registers (item
-                                kernel); 1 rows staged by bulk copies into a shared-
-                                memory ring (warp-specialised kernel); 2 rows streamed
-                                by every thread into a cp.async ring (streaming kernel) */
+                                kernel); 2 rows streamed by every thread into a
+                                cp.async ring (streaming kernel) */
     int32_t cluster;         /* rms: CTAs per row (cluster size); else 1 */
     int32_t block;           /* threads per CTA */
     int32_t direct_angles;   /* rope: 1 if each work item read its (cos, sin) straight
@@ -398,16 +402,15 @@ qkr_status qkr_last_launch(qkr_launch_info *info);
 qkr_status qkr_launch_overlap(int32_t enable);
 
 /* Launch-shape override for the rope kernels, for tuning sweeps.  pipeline:
- * 0 automatic, 1 item kernel (rows straight into registers), 2 bulk-copy
- * pipelined kernel, 3 streaming kernel (cp.async row ring); calls a forced
- * kernel cannot serve fail with QKR_ERR_CUDA.  heads per work item (1..4; the
- * streaming kernel takes 1, 2 or 4), tokens per CTA or per pipeline tile
- * (1..64; kernels that stage angles cap it by their shared memory) and ring
- * depth of the streaming kernel (2..4); 0 keeps the automatic choice.
- * Process-wide; a launch racing a change on another thread takes the old or
- * the new value of each knob.  Every shape computes bit-identical results: a row's
- * arithmetic does not depend on it.  Returns QKR_ERR_INVALID_ARG out of
- * range. */
+ * 0 automatic, 1 item kernel (rows straight into registers), 3 streaming
+ * kernel (cp.async row ring); calls a forced kernel cannot serve fail with
+ * QKR_ERR_CUDA.  heads per work item (1..4; the streaming kernel takes 1, 2 or
+ * 4), tokens per CTA (1..64; kernels that stage angles cap it by their shared
+ * memory) and ring depth of the streaming kernel (2..4; 1 counts as 2); 0
+ * keeps the automatic choice.  Process-wide; a launch racing a change on
+ * another thread takes the old or the new value of each knob.  Every shape
+ * computes bit-identical results: a row's arithmetic does not depend on it.
+ * Returns QKR_ERR_INVALID_ARG out of range. */
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,
                          int32_t stages);
 
@@ -428,12 +431,25 @@ qkr_status qkr_tune_rope_lanes(int32_t lanes);
 qkr_status qkr_tune_rms(int32_t cluster);
 
 /* Device status word of the library on the current device (0 = healthy).
- * Kernels that wait on shared-memory barriers give every wait a time budget;
- * a wait that runs out sets a bit here (1: producer, 2: consumer) and the
- * kernel returns early instead of hanging.  Bit 4: rope_set_rows met a row
- * index outside the cache (that row was not written).  Synchronous (copies
- * the word to the host); reset != 0 clears it.  Not for the hot path. */
+ * Bit 4: rope_set_rows met a row index outside the cache (that row was not
+ * written).  The word is shared by every call of the process on that device,
+ * so a bit cannot be traced to the call that raised it; it stays set until a
+ * read with reset != 0 clears it.  The read (and the clear) is one atomic
+ * exchange on the device, ordered after the work of every blocking stream:
+ * a bit raised concurrently by a kernel on a non-blocking stream is returned
+ * by this read or by the next, never lost.  Synchronous (copies the word to
+ * the host); concurrent reads from several host threads are serialised.  Not
+ * for the hot path. */
 qkr_status qkr_device_status(uint32_t *status, int32_t reset);
+
+/* The launch floor, for measurement: enqueues one kernel of `grid` CTAs of
+ * `block` threads (a multiple of 32, at most 1024) that does nothing but the
+ * programmatic-launch wait and trigger every library kernel begins with,
+ * launched with the same attributes (qkr_launch_overlap).  Back-to-back
+ * launches of it show the per-launch cost no kernel of this library can go
+ * below (vllm.cpp #185 measures its decode RMSNorm per call; a call that
+ * moves kilobytes costs what a launch costs).  Touches no memory. */
+qkr_status qkr_null_launch(void *stream, int64_t grid, int32_t block);
 
 /* Writes the axis (0 t, 1 h, 2 w, 3 e) of pairs 0..P-1 under a section mode
  * to axis_out (device int8 [P]) with the kernels' own section rule.

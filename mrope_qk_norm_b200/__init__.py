@@ -25,12 +25,12 @@ ANGLE_POSITIONS, ANGLE_TABLE = 0, 1
 FLAG_ROUND_NORMALIZED_BF16 = 1
 KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange",
                 4: "vit_setup", 5: "rms_rows", 6: "rms_cluster", 7: "section_map",
-                8: "vit_positions"}
+                8: "vit_positions", 9: "null"}
 
 EXPORTS = ("fused_qk_norm_rope", "fused_qkv_norm_rope", "mrope_apply", "rope_set_rows",
            "vit_mrope_setup", "rms_norm_residual", "rms_norm_fp8", "qkr_last_error", "qkr_version", "qkr_last_launch", "qkr_section_map",
            "qkr_vit_positions", "qkr_tune_rope", "qkr_tune_rope_lanes", "qkr_tune_rms", "qkr_device_status",
-           "qkr_launch_overlap")
+           "qkr_launch_overlap", "qkr_null_launch")
 
 
 class QkrError(RuntimeError):
@@ -97,6 +97,7 @@ def _load() -> ctypes.CDLL:
         "qkr_tune_rms": [I32],
         "qkr_launch_overlap": [I32],
         "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
+        "qkr_null_launch": [V, I64, I32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -182,6 +183,11 @@ def tune_rms(cluster: int = 0) -> None:
 def launch_overlap(enable: bool) -> None:
     """Programmatic dependent launch for every kernel of the library (default on)."""
     _check(_lib.qkr_launch_overlap(1 if enable else 0))
+
+
+def null_launch(grid: int = 1, block: int = 128, stream=None) -> None:
+    """The launch-floor probe: an empty kernel with the library's launch attributes."""
+    _check(_lib.qkr_null_launch(_stream(stream), grid, block))
 
 
 def device_status(reset: bool = False) -> int:

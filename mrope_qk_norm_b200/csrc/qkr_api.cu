@@ -5,6 +5,7 @@
 // allocates, frees or synchronises.
 
 #include <atomic>
+#include <climits>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -64,6 +65,36 @@ Span view_span(const void *base, int64_t T, int64_t ts, int64_t H, int64_t hs, i
 bool overlap(const Span &a, const Span &b)
 {
     return a.lo < a.hi && b.lo < b.hi && a.lo < b.hi && b.lo < a.hi;
+}
+
+// A strided bf16 [T, H, D] view: element (t, h, d) at base + t*ts + h*hs + d.
+struct View {
+    const void *base = nullptr;
+    int64_t T = 0, ts = 0, H = 0, hs = 0, D = 0;
+};
+Span span(const View &v) { return view_span(v.base, v.T, v.ts, v.H, v.hs, v.D); }
+
+// True when two views share no element.  Either their byte spans do not
+// intersect, or both advance by the same token stride and, within that
+// stride, the columns one view's token row covers lie outside the other's
+// (Q and K as column windows of one packed [T, 3, H, D] buffer, say): then no
+// row of one reaches a byte of the other, whatever tokens they cover.
+bool views_disjoint(const View &a, const View &b)
+{
+    const Span sa = span(a), sb = span(b);
+    if (!overlap(sa, sb))
+        return true;
+    if (a.ts != b.ts || a.ts <= 0)
+        return false;
+    const int64_t TS = 2 * a.ts;                        // token stride in bytes
+    const int64_t wa = 2 * ((a.H - 1) * a.hs + a.D);    // bytes of a token row
+    const int64_t wb = 2 * ((b.H - 1) * b.hs + b.D);
+    if (wa > TS || wb > TS)
+        return false;
+    const int64_t diff = (int64_t)(reinterpret_cast<uintptr_t>(b.base) -
+                                   reinterpret_cast<uintptr_t>(a.base));
+    const int64_t rel = ((diff % TS) + TS) % TS;        // b's row start inside a's row grid
+    return rel >= wa && rel + wb <= TS;
 }
 
 // Largest element offset a view reaches must stay far from int64 overflow.
@@ -331,39 +362,40 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     if (!view_fits(T, qo_ts, 1, 0, Hq * D) || !view_fits(k_rows_out, ko_ts, 1, 0, Hk * D))
         return fail(QKR_ERR_INVALID_ARG, "output view exceeds the address range");
 
-    // Aliasing: outputs may equal inputs only where allowed, never overlap otherwise.
-    const Span so_q = view_span(q_out, T, qo_ts, Hq, D, D);
-    const Span so_k = view_span(k_out, k_rows_out, ko_ts, Hk, D, D);
-    if (overlap(so_q, so_k))
+    // Aliasing: outputs may equal inputs only where allowed (exact in-place),
+    // and must share no element with any other view.
+    const View vo_q{q_out, T, qo_ts, Hq, D, D};
+    const View vo_k{k_out, k_rows_out, ko_ts, Hk, D, D};
+    if (!views_disjoint(vo_q, vo_k))
         return fail(QKR_ERR_UNSUPPORTED, "q_out and k_out overlap");
-    Span so_v;
+    View vo_v;
     if (Hv > 0) {
         if (!view_fits(T, vo_ts, 1, 0, Hv * D))
             return fail(QKR_ERR_INVALID_ARG, "v_out view exceeds the address range");
-        so_v = view_span(v_out, T, vo_ts, Hv, D, D);
-        if (overlap(so_v, so_q) || overlap(so_v, so_k))
+        vo_v = View{v_out, T, vo_ts, Hv, D, D};
+        if (!views_disjoint(vo_v, vo_q) || !views_disjoint(vo_v, vo_k))
             return fail(QKR_ERR_UNSUPPORTED, "v_out overlaps q_out or k_out");
     }
     for (int s = 0; s < n_streams; ++s) {
         const qkr_stream_desc &d = streams[s];
         if (d.n_tokens == 0)
             continue;
-        const Span si_q = view_span(qb[s], d.n_tokens, d.q_tok_stride, Hq, d.q_head_stride, D);
-        const Span si_k = view_span(kb[s], d.n_tokens, d.k_tok_stride, Hk, d.k_head_stride, D);
+        const View vi_q{qb[s], d.n_tokens, d.q_tok_stride, Hq, d.q_head_stride, D};
+        const View vi_k{kb[s], d.n_tokens, d.k_tok_stride, Hk, d.k_head_stride, D};
         const bool q_same = inplace_ok && n_streams == 1 && qb[s] == q_out &&
                             d.q_tok_stride == qo_ts && d.q_head_stride == D;
         const bool k_same = inplace_ok && n_streams == 1 && kb[s] == k_out &&
                             d.k_tok_stride == ko_ts && d.k_head_stride == D;
-        if ((overlap(so_q, si_q) && !q_same) || overlap(so_q, si_k) ||
-            (overlap(so_k, si_k) && !k_same) || overlap(so_k, si_q))
+        if ((!views_disjoint(vo_q, vi_q) && !q_same) || !views_disjoint(vo_q, vi_k) ||
+            (!views_disjoint(vo_k, vi_k) && !k_same) || !views_disjoint(vo_k, vi_q))
             return fail(QKR_ERR_UNSUPPORTED,
                         inplace_ok ? "outputs overlap inputs (only exact in-place is allowed)"
                                    : "outputs must not overlap the inputs (fresh outputs)");
         if (Hv > 0) {
-            const Span si_v =
-                view_span(vb[s], d.n_tokens, d.v_tok_stride, Hv, d.v_head_stride, D);
-            if (overlap(so_v, si_q) || overlap(so_v, si_k) || overlap(so_v, si_v) ||
-                overlap(so_q, si_v) || overlap(so_k, si_v))
+            const View vi_v{vb[s], d.n_tokens, d.v_tok_stride, Hv, d.v_head_stride, D};
+            if (!views_disjoint(vo_v, vi_q) || !views_disjoint(vo_v, vi_k) ||
+                !views_disjoint(vo_v, vi_v) || !views_disjoint(vo_q, vi_v) ||
+                !views_disjoint(vo_k, vi_v))
                 return fail(QKR_ERR_UNSUPPORTED,
                             "outputs must not overlap the inputs (fresh outputs)");
         }
@@ -471,14 +503,28 @@ qkr_status qkr_tune_rope_lanes(int32_t lanes)
 qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t tokens_per_cta,
                          int32_t stages)
 {
-    if (pipeline < 0 || pipeline > 3 || heads_per_item < 0 || heads_per_item > 4 ||
-        tokens_per_cta < 0 || tokens_per_cta > 64 || stages < 0 || stages == 1 || stages > 4)
+    if ((pipeline != 0 && pipeline != 1 && pipeline != 3) || heads_per_item < 0 ||
+        heads_per_item > 4 || tokens_per_cta < 0 || tokens_per_cta > 64 || stages < 0 ||
+        stages > 4)
         return fail(QKR_ERR_INVALID_ARG,
-                    "pipeline in [0, 3], heads_per_item in [0, 4], tokens_per_cta in [0, 64], "
-                    "stages 0 or in [2, 4]");
+                    "pipeline 0, 1 or 3, heads_per_item in [0, 4], tokens_per_cta in [0, 64], "
+                    "stages in [0, 4]");
     qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta, stages);
     g_error.clear();
     return QKR_OK;
+}
+
+qkr_status qkr_null_launch(void *stream, int64_t grid, int32_t block)
+{
+    if (grid < 1 || grid > INT32_MAX || block < 32 || block > 1024 || block % 32)
+        return fail(QKR_ERR_INVALID_ARG, "grid in [1, 2^31), block a multiple of 32 in [32, 1024]");
+    qkr::LaunchRecord rec;
+    qkr_status r = cuda_result(qkr::launch_null(grid, block, static_cast<cudaStream_t>(stream),
+                                                &rec),
+                               "null kernel launch");
+    if (r == QKR_OK)
+        g_last = rec;
+    return r;
 }
 
 qkr_status qkr_device_status(uint32_t *status, int32_t reset)

@@ -190,21 +190,20 @@ struct LaunchRecord {
 };
 
 // Launch-shape override of the rope kernels (0: automatic); pipeline: 0 auto,
-// 1 item kernel only, 2 bulk-copy pipelined kernel only, 3 streaming kernel only.
+// 1 item kernel only, 3 streaming kernel only; stages: passes of the streaming
+// kernel's row ring.
 void set_rope_shape_override(int pipeline, int heads_per_item, int tokens_per_cta,
                              int stages);
 // Lanes per head row of the GPT-J (VECTOR) layout, for tuning (0: automatic).
 void set_rope_lanes_override(int lanes);
 
-// Bulk-copy pipelined rope kernel (rope_tma.cu); cudaErrorNotSupported when a
-// call is outside what it serves.
-cudaError_t launch_rope_tma(const RopeParams &p, int layout_paired, int lpr, int ns,
-                            int tokens_per_tile, cudaStream_t stream, LaunchRecord *rec);
-// Reads (and optionally clears) the device status word that bounded waits set
-// on timeout.  Synchronous.
+// Reads (and optionally clears, in one atomic step on the device) the device
+// status word that kernels raise bits in (status.cu).  Synchronous.
 cudaError_t read_device_status(unsigned *status, bool reset);
 // Device address of that status word on the current device.
 cudaError_t device_status_address(unsigned **addr);
+// The launch-floor probe: an empty kernel with the library's launch attributes.
+cudaError_t launch_null(int64_t grid, int block, cudaStream_t stream, LaunchRecord *rec);
 
 // Each launcher enqueues exactly one kernel and returns the CUDA launch status.
 cudaError_t launch_rope_rows(const RopeParams &p, int pairing, cudaStream_t stream,

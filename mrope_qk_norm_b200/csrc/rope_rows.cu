@@ -171,7 +171,7 @@ KernelFn pick_exchange(int lpr, int ns)
 
 // Process-wide tuning overrides (atomics: a knob set from one thread while
 // another launches is a race on the launch shape only, never on memory).
-std::atomic<int> g_force_pipe{0};  // 0 automatic, 1 item, 2 bulk-copy, 3 streaming kernel
+std::atomic<int> g_force_pipe{0};  // 0 automatic, 1 item, 3 streaming kernel
 std::atomic<int> g_force_u{0};     // heads per item (0: automatic)
 std::atomic<int> g_force_tt{0};    // tokens per CTA (0: automatic)
 std::atomic<int> g_force_s{0};     // streaming ring depth (0: automatic)
@@ -261,7 +261,7 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
     int u = fu > 0 ? fu : 2;
     if (u == 3)
         u = 2;
-    const int S = fs > 0 ? fs : 2;
+    const int S = fs > 1 ? fs : 2;
     p.stages = S;
     p.pw = layout == VECTOR ? p.D / 2 : p.P;
     const int cs_ld = (p.pw + 3) & ~3;
@@ -385,11 +385,6 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
             lpr = g_force_lpr;
         ns = (nvec + lpr - 1) / lpr;
     }
-    // The bulk-copy pipelined kernel (rope_tma.cu) is selected explicitly: it
-    // measured slower than the item kernel, which reaches ~90% of a plain
-    // elementwise streaming pass over the same bytes.
-    if (layout != EXCHANGE && g_force_pipe == 2)
-        return launch_rope_tma(p, layout == PAIRED, lpr, ns, g_force_tt, stream, rec);
     if (p.T > INT_MAX)
         return cudaErrorInvalidConfiguration;
     // Angles from positions: the streaming kernel (sincosf once per token of a

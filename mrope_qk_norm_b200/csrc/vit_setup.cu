@@ -3,15 +3,14 @@
 // expose the section rule and the grid-to-position mapping to the tests.
 //
 // B200 mapping.  The setup writes 2 * 4 bytes per (token, section column),
-// computing one sincosf per cell; it is latency- and launch-bound at these
-// sizes (8 MB for 16k tokens).  A CTA covers kTokens tokens.  It first stages
-// the grid metadata (cu_seqlens, grids) and inv_freq in shared memory with
-// independent loads -- one memory round trip instead of the binary search's
-// chain of dependent loads -- then one thread per token derives (t, h, w)
-// into shared memory, and each thread keeps one column (axis, offset and
-// inv_freq fixed in registers) while walking the tokens, consecutive threads
-// on consecutive columns so each warp's stores are contiguous.
-
+// computing one sincosf per cell; at these sizes (8 MB for 16k tokens) it is
+// bound by launch latency and by the sincosf issue rate, not by bytes.  So
+// every warp works on its own, with no block barrier: a warp owns 8
+// consecutive tokens; lanes 0..7 derive one token's (t, h, w) each (the grid
+// found by shuffles over a register copy of the grid boundaries when there
+// are at most 32 grids), the positions are broadcast by shuffle, and each
+// lane owns one column of every 32 (its axis, section offset and inv_freq
+// fixed for the pass), so a warp's stores to a token row are contiguous.
 #include <climits>
 
 #include "qkr_internal.cuh"
@@ -19,35 +18,22 @@
 namespace qkr {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTokens = 32;
-constexpr int kSmemGrids = 512;  // grids whose metadata a CTA stages in shared memory
-constexpr int kMaxVitPairs = 512;  // per-axis inv_freq lengths staged in shared memory
+constexpr int kThreads = 256;     // debug kernels
+constexpr int kVitWarps = 4;      // warps per setup CTA
+constexpr int kVitTokPerWarp = 8; // tokens one warp writes
+constexpr int kVitThreads = 32 * kVitWarps;
+constexpr int kTokens = kVitWarps * kVitTokPerWarp;  // tokens per setup CTA
 
-// (t, h, w) of token n (cu / grids in shared or global memory).  The grid is
-// the g with cu[g] <= n < cu[g+1]
-// (binary search over the nondecreasing boundaries; empty grids are never
-// selected).  Inside a frame of h*w tokens, tokens come in m x m merge blocks
-// in row-major block order, each block's patches in row-major order.
-__device__ __forceinline__ void token_position(const int32_t *cu, const int32_t *grids, int G,
-                                               int64_t n, int m, int &tp, int &hp, int &wp)
+// (t, h, w) of the token at `local` index inside a grid of [., h, w] with
+// merge size m.  Inside a frame of h*w tokens, tokens come in m x m merge
+// blocks in row-major block order, each block's patches in row-major order.
+__device__ __forceinline__ void grid_position(int64_t local, int h, int w, int m, int &tp,
+                                              int &hp, int &wp)
 {
-    int lo = 0, hi = G;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if ((int64_t)cu[mid + 1] <= n)
-            lo = mid + 1;
-        else
-            hi = mid;
-    }
-    const int g = lo < G ? lo : G - 1;
-    const int64_t local = n - (int64_t)cu[g];
-    const int h = grids[3 * g + 1];
-    const int w = grids[3 * g + 2];
     const int64_t frame = max((int64_t)h * w, (int64_t)1);
     if (frame <= 0xffffffffLL && local >= 0 && local <= 0xffffffffLL && m > 0) {
         // the usual case, in 32-bit unsigned arithmetic (a 64-bit division is
-        // several times longer, and this chain is the CTA's critical path)
+        // several times longer)
         const uint32_t l32 = (uint32_t)local, f32 = (uint32_t)frame, mm = (uint32_t)(m * m);
         const uint32_t t32 = l32 / f32;
         const uint32_t in_frame = l32 - t32 * f32;
@@ -73,80 +59,84 @@ __device__ __forceinline__ void token_position(const int32_t *cu, const int32_t 
     wp = (int)(bcol * m + patch % m);
 }
 
-__global__ void __launch_bounds__(kThreads) vit_setup_kernel(const __grid_constant__ VitParams p)
+// (t, h, w) of token n: the grid is the g with cu[g] <= n < cu[g+1] (binary
+// search over the nondecreasing boundaries; empty grids are never selected).
+__device__ __forceinline__ void token_position(const int32_t *cu, const int32_t *grids, int G,
+                                               int64_t n, int m, int &tp, int &hp, int &wp)
+{
+    int lo = 0, hi = G;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((int64_t)__ldg(cu + mid + 1) <= n)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    const int g = lo < G ? lo : G - 1;
+    grid_position(n - (int64_t)__ldg(cu + g), __ldg(grids + 3 * g + 1), __ldg(grids + 3 * g + 2),
+                  m, tp, hp, wp);
+}
+
+__global__ void __launch_bounds__(kVitThreads)
+vit_setup_kernel(const __grid_constant__ VitParams p)
 {
     pdl_wait();
     pdl_trigger();
-    __shared__ int spos[3][kTokens];
-    __shared__ int32_t scu[kSmemGrids + 1];
-    __shared__ int32_t sgrid[3 * kSmemGrids];
-    __shared__ float sinv[3][kMaxVitPairs];
-    // Stage the grid metadata and inv_freq with independent loads (one DRAM
-    // round trip) instead of the binary search's chain of dependent loads.
-    const bool staged = p.G <= kSmemGrids;
-    if (staged) {
-        for (int i = threadIdx.x; i <= p.G; i += kThreads)
-            scu[i] = __ldg(p.cu + i);
-        for (int i = threadIdx.x; i < 3 * p.G; i += kThreads)
-            sgrid[i] = __ldg(p.grids + i);
-    }
-    const bool inv_staged =
-        p.half[0] <= kMaxVitPairs && p.half[1] <= kMaxVitPairs && p.half[2] <= kMaxVitPairs;
-    if (inv_staged)
-        for (int a = 0; a < 3; ++a)
-            for (int i = threadIdx.x; i < p.half[a]; i += kThreads)
-                sinv[a][i] = __ldg(p.inv[a] + i);
-    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t n0 = ((int64_t)blockIdx.x * kVitWarps + warp) * kVitTokPerWarp;
+    if (n0 >= p.N)
+        return;  // warp-uniform
+    const int ntok = (int)min((int64_t)kVitTokPerWarp, p.N - n0);
 
-    const int64_t n0 = (int64_t)blockIdx.x * kTokens;
-    const int ntok = (int)min((int64_t)kTokens, p.N - n0);
-    if (threadIdx.x < ntok) {
-        int tp, hp, wp;
-        token_position(staged ? scu : p.cu, staged ? sgrid : p.grids, p.G, n0 + threadIdx.x,
-                       p.m, tp, hp, wp);
-        spos[0][threadIdx.x] = tp;
-        spos[1][threadIdx.x] = hp;
-        spos[2][threadIdx.x] = wp;
+    // Lane j < ntok derives the position of token n0 + j (other lanes repeat
+    // the last token, so every lane runs the same code).
+    const int64_t n = n0 + min(lane, ntok - 1);
+    int tp, hp, wp;
+    if (p.G <= 32) {
+        // lane l holds grid l's boundaries and sizes: one load each, and the
+        // grid of a token is the number of grids that end at or before it
+        const bool have = lane < p.G;
+        const int32_t end_l = have ? __ldg(p.cu + lane + 1) : 0;
+        const int32_t start_l = have ? __ldg(p.cu + lane) : 0;
+        const int32_t h_l = have ? __ldg(p.grids + 3 * lane + 1) : 1;
+        const int32_t w_l = have ? __ldg(p.grids + 3 * lane + 2) : 1;
+        int g = 0;
+        for (int k = 0; k < p.G; ++k)  // uniform trip count
+            g += (int64_t)__shfl_sync(0xffffffffu, end_l, k) <= n ? 1 : 0;
+        g = min(g, p.G - 1);
+        const int32_t start = __shfl_sync(0xffffffffu, start_l, g);
+        const int32_t h = __shfl_sync(0xffffffffu, h_l, g);
+        const int32_t w = __shfl_sync(0xffffffffu, w_l, g);
+        grid_position(n - (int64_t)start, h, w, p.m, tp, hp, wp);
+    } else {
+        token_position(p.cu, p.grids, p.G, n, p.m, tp, hp, wp);
     }
-    __syncthreads();
 
     const int P = p.P;
     const int end_t = p.half[0], end_h = p.half[0] + p.half[1];
-    if (P <= kThreads) {
-        // A thread owns one column for the whole pass: its axis, section
-        // offset and inv_freq are fixed, and it walks the CTA's tokens with
-        // a stride of kThreads / P (consecutive threads on consecutive
-        // columns of one token row, so each warp's stores are contiguous).
-        const int tpp = kThreads / P;
-        const int col = threadIdx.x % P;
-        const int tsub = threadIdx.x / P;
-        if (tsub < tpp) {
-            const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
-            const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
-            const float f = inv_staged ? sinv[axis][col - off] : __ldg(p.inv[axis] + (col - off));
-            const int64_t base = ((int64_t)axis * p.N + n0) * P + col;
+    for (int c0 = 0; c0 < P; c0 += 32) {  // uniform trip count
+        // this lane's column of the pass: its axis, offset and inv_freq
+        const int col = c0 + lane;
+        const bool live = col < P;
+        const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
+        const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
+        const float f = live ? __ldg(p.inv[axis] + (col - off)) : 0.f;
+        float *cdst = p.cos_out + ((int64_t)axis * p.N + n0) * P + col;
+        float *sdst = p.sin_out + ((int64_t)axis * p.N + n0) * P + col;
 #pragma unroll 4
-            for (int tt = tsub; tt < ntok; tt += tpp) {
-                const float theta = __fmul_rn((float)spos[axis][tt], f);
-                float s, c;
-                sincosf(theta, &s, &c);
-                __stcs(p.cos_out + base + (int64_t)tt * P, c);
-                __stcs(p.sin_out + base + (int64_t)tt * P, s);
+        for (int j = 0; j < ntok; ++j) {  // uniform trip count
+            const int pt = __shfl_sync(0xffffffffu, tp, j);
+            const int ph = __shfl_sync(0xffffffffu, hp, j);
+            const int pw = __shfl_sync(0xffffffffu, wp, j);
+            const int pos = axis == 0 ? pt : (axis == 1 ? ph : pw);
+            const float theta = __fmul_rn((float)pos, f);
+            float sv, cv;
+            sincosf(theta, &sv, &cv);
+            if (live) {
+                __stcs(cdst + (int64_t)j * P, cv);
+                __stcs(sdst + (int64_t)j * P, sv);
             }
-        }
-    } else {
-        for (int idx = threadIdx.x; idx < ntok * P; idx += kThreads) {
-            const int tt = idx / P;
-            const int col = idx - tt * P;
-            const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
-            const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
-            const float f = inv_staged ? sinv[axis][col - off] : __ldg(p.inv[axis] + (col - off));
-            const float theta = __fmul_rn((float)spos[axis][tt], f);
-            float s, c;
-            sincosf(theta, &s, &c);
-            const int64_t at = ((int64_t)axis * p.N + n0 + tt) * P + col;
-            __stcs(p.cos_out + at, c);
-            __stcs(p.sin_out + at, s);
         }
     }
 }
@@ -187,13 +177,13 @@ cudaError_t launch_vit_setup(const VitParams &p, cudaStream_t stream, LaunchReco
     const int64_t grid = (p.N + kTokens - 1) / kTokens;
     if (grid > INT_MAX)
         return cudaErrorInvalidConfiguration;
-    cudaError_t err = launch(vit_setup_kernel, dim3((unsigned)grid), dim3(kThreads), 0, stream,
-                             1, p);
+    cudaError_t err = launch(vit_setup_kernel, dim3((unsigned)grid), dim3(kVitThreads), 0,
+                             stream, 1, p);
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();
         rec->kernel = QKR_KERNEL_VIT_SETUP;
         rec->tokens_per_cta = kTokens;
-        rec->block = kThreads;
+        rec->block = kVitThreads;
         rec->grid = grid;
         rec->launches = 1;
     }

@@ -204,7 +204,9 @@ def test_launch_switch_refusals(qkr):
     assert L.qkr_launch_overlap(2) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_launch_overlap(-1) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(4, 0, 0, 0) == qkr.QKR_ERR_INVALID_ARG
-    assert L.qkr_tune_rope(3, 0, 0, 1) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(2, 0, 0, 0) == qkr.QKR_ERR_INVALID_ARG   # no bulk-copy kernel
+    assert L.qkr_tune_rope(3, 0, 0, 5) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(1, 0, 0, -1) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(3, 5, 0, 0) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(3, 0, 65, 0) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(0, 0, 0, 0) == qkr.QKR_OK
@@ -262,3 +264,27 @@ def test_too_many_tokens_is_refused_not_launched(qkr):
     st = L.fused_qk_norm_rope(None, arr, 1, FAKE + (5 << 40), FAKE + (6 << 40), 64, 64, 1, 1, 64,
                               64, 0, 1e-6, ctypes.byref(a), 0)
     assert st == qkr.QKR_ERR_UNSUPPORTED and "2^31" in _err(qkr)
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="an accepted call would launch on the fake addresses")
+def test_packed_qkv_in_place_passes_validation(qkr):
+    """Q and K as column windows of one packed [T, 3, H, D] buffer, rotated in
+    place: their byte ranges interleave but share no element, so the host
+    accepts the call (here it then fails only at the launch, with no device);
+    windows that do share elements are still refused."""
+    T, H, D = 4, 2, 64
+    ts = 3 * H * D
+    base = FAKE
+    q, k = base, base + 2 * H * D          # columns [0, HD) and [HD, 2HD) of each token row
+    st = _mrope(qkr, q=q, k=k, q_out=q, k_out=k, T=T, Hq=H, Hkv=H, D=D, rot=D, qts=ts, kts=ts,
+                qots=ts, kots=ts, T_total=T, sec=(16, 8, 8, 0))
+    assert st == qkr.QKR_ERR_CUDA, _err(qkr)   # validation passed; no device to launch on
+    # K window shifted by 8 elements into Q's columns: shared elements, refused
+    st = _mrope(qkr, q=q, k=q + 2 * (H * D - 8), q_out=q, k_out=q + 2 * (H * D - 8), T=T, Hq=H,
+                Hkv=H, D=D, rot=D, qts=ts, kts=ts, qots=ts, kots=ts, T_total=T, sec=(16, 8, 8, 0))
+    assert st == qkr.QKR_ERR_UNSUPPORTED
+    # an output window laid over the other input's columns: refused
+    st = _mrope(qkr, q=q, k=k, q_out=k, k_out=q, T=T, Hq=H, Hkv=H, D=D, rot=D, qts=ts, kts=ts,
+                qots=ts, kots=ts, T_total=T, sec=(16, 8, 8, 0))
+    assert st == qkr.QKR_ERR_UNSUPPORTED

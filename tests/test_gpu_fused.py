@@ -3,9 +3,10 @@
 Covers the single-stream configuration (T=16, H=4, D=64, NeoX, positions
 0..15, seed 0), the joint text/image configuration at full size (512 + 4096
 tokens, 24 heads, D=128, fp32 [4608, 64] cos/sin table, both pairings), the
-2^31-element storage-offset variant on either stream, strided views, the
-bf16-rounded-normalised-value contract, every kernel layout and ragged
-shapes.
+2^31-element storage-offset variant on either stream at full size (and row
+offsets past 2^31 formed inside the kernel), strided views, the
+bf16-rounded-normalised-value contract, every kernel layout, launch shape
+and ragged shapes.
 """
 import numpy as np
 import pytest
@@ -89,40 +90,100 @@ def test_joint_small_ragged_vs_oracle():
         check_against_oracle(w, what="joint small")
 
 
-@pytest.mark.parametrize("which", [0, 1])
-@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
-def test_large_storage_offset(which, pairing):
-    """One stream lives 2^31 elements into its storage (needs > 8 GiB free)."""
-    free, _ = torch.cuda.mem_get_info()
-    if free < 12 * 2 ** 30:
-        pytest.skip("needs 12 GiB of free device memory")
-    w = W.config3(seed=17, T_txt=64, img_h=16, img_w=16, H=24, D=128, pairing=pairing)
-    ref_q, ref_k = run_fused(w)
+def _offset_stream(q, k, off):
+    """Copies of q and k placed `off` elements into fresh storage."""
+    big_q = torch.empty(off + q.numel(), dtype=torch.bfloat16, device="cuda")
+    big_q[off:].copy_(q.reshape(-1))
+    big_k = torch.empty(off + k.numel(), dtype=torch.bfloat16, device="cuda")
+    big_k[off:].copy_(k.reshape(-1))
+    qv, kv = big_q[off:].view(q.shape), big_k[off:].view(k.shape)
+    assert qv.storage_offset() == off and kv.storage_offset() == off
+    return qv, kv, [big_q, big_k]
+
+
+def _wide_row_stream(q, k, ts):
+    """q and k as the first two column windows of one buffer whose token rows
+    are `ts` elements apart, so token t of the stream sits t*ts elements into
+    the storage."""
+    T, H, D = q.shape
+    buf = torch.empty(T, ts, dtype=torch.bfloat16, device="cuda")
+    buf[:, :H * D].copy_(q.reshape(T, H * D))
+    buf[:, H * D:2 * H * D].copy_(k.reshape(T, H * D))
+    qv = buf[:, :H * D].view(T, H, D)
+    kv = buf[:, H * D:2 * H * D].view(T, H, D)
+    assert qv.stride(0) == ts and kv.stride(0) == ts
+    return qv, kv, [buf]
+
+
+def _run_joint_with(w, which, place):
+    """The joint launch with stream `which` placed by `place(q, k)`."""
     keep, streams = [], []
-    off = 2 ** 31
     for i, s in enumerate(w.streams):
         q, k = to_dev(s.q), to_dev(s.k)
         if i == which:
-            big_q = torch.empty(off + q.numel(), dtype=torch.bfloat16, device="cuda")
-            big_q[off:].copy_(q.reshape(-1))
-            big_k = torch.empty(off + k.numel(), dtype=torch.bfloat16, device="cuda")
-            big_k[off:].copy_(k.reshape(-1))
-            q = big_q[off:].view(q.shape)
-            k = big_k[off:].view(k.shape)
-            assert q.storage_offset() == off
-            keep += [big_q, big_k]
+            q, k, big = place(q, k)
+            keep += big
         gq, gk = to_dev(s.gamma_q), to_dev(s.gamma_k)
         keep += [q, k, gq, gk]
         streams.append((q, k, gq, gk))
     T = w.n_tokens
-    qo = torch.empty(T, w.Hq, w.D, dtype=torch.bfloat16, device="cuda")
-    ko = torch.empty(T, w.Hk, w.D, dtype=torch.bfloat16, device="cuda")
+    qo = Guarded((T, w.Hq, w.D))
+    ko = Guarded((T, w.Hk, w.D))
     a = _angle_desc(w.angle, keep)
-    qkr.fused_qk_norm_rope(streams, qo, ko, w.rot, w.pairing, w.eps, a)
+    qkr.fused_qk_norm_rope(streams, qo.tensor, ko.tensor, w.rot, w.pairing, w.eps, a)
     torch.cuda.synchronize()
-    assert torch.equal(qo.view(torch.int16), ref_q.view(torch.int16))
-    assert torch.equal(ko.view(torch.int16), ref_k.view(torch.int16))
+    qo.check()
+    ko.check()
     del keep
+    return qo.tensor, ko.tensor
+
+
+@pytest.mark.parametrize("which", [0, 1])
+@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
+def test_large_storage_offset_full_size(which, pairing):
+    """The joint workload at full size (512 + 4096 tokens, 24 heads, D=128)
+    with one stream 2^31 elements into its storage (vllm-omni #7600, 64-bit
+    row addressing): equal bit for bit to the launch without the offset and
+    within tolerance of the oracle.  Needs about 8.1 GiB for the offset
+    stream."""
+    free, _ = torch.cuda.mem_get_info()
+    if free < 12 * 2 ** 30:
+        pytest.skip("needs 12 GiB of free device memory")
+    w = W.config3(pairing=pairing)
+    assert w.n_tokens == 4608 and w.Hq == 24 and w.D == 128
+    ref_q, ref_k = run_fused(w)
+    q, k = _run_joint_with(w, which, lambda q, k: _offset_stream(q, k, 2 ** 31))
+    assert torch.equal(q.view(torch.int16), ref_q.view(torch.int16))
+    assert torch.equal(k.view(torch.int16), ref_k.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(q, rq, "offset q")
+    assert_bf16_close(k, rk, "offset k")
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("which", [0, 1])
+@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
+def test_row_offsets_past_2_31_in_kernel(which, pairing):
+    """The kernel's own row addressing past 2^31 elements: the stream's token
+    stride is so wide that token t*stride crosses 2^31 inside the launch
+    (the storage offset above is added on the host; here the kernel forms
+    the large offsets).  Full-size joint workload; about 4.4 GiB for the wide
+    stream."""
+    free, _ = torch.cuda.mem_get_info()
+    if free < 10 * 2 ** 30:
+        pytest.skip("needs 10 GiB of free device memory")
+    w = W.config3(pairing=pairing)
+    T_s = int(w.streams[which].q.shape[0])
+    ts = -(-(2 ** 31 + 2 ** 20) // (T_s - 1))
+    ts = -(-ts // 8) * 8                      # a multiple of 8 elements
+    assert (T_s - 1) * ts > 2 ** 31
+    ref_q, ref_k = run_fused(w)
+    q, k = _run_joint_with(w, which, lambda q, k: _wide_row_stream(q, k, ts))
+    assert torch.equal(q.view(torch.int16), ref_q.view(torch.int16))
+    assert torch.equal(k.view(torch.int16), ref_k.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(q, rq, "wide-row q")
+    assert_bf16_close(k, rk, "wide-row k")
     torch.cuda.empty_cache()
 
 
@@ -210,50 +271,57 @@ def test_empty_streams():
     assert qkr.last_launch()["launches"] == 0
 
 
-def _both_kernels(w, flags=0):
-    """Run once with the bulk-copy pipelined kernel and once with the register
-    kernel; return both results and the two launch records."""
+def _shape_variants(w, flags=0):
+    """Run the item kernel at every heads-per-item choice and the streaming
+    kernel; return the results and launch records."""
+    outs = []
     try:
-        qkr.tune_rope(2, 0, 0)
-        a = run_fused(w, flags)
-        ia = qkr.last_launch()
-        qkr.tune_rope(1, 0, 0)
-        b = run_fused(w, flags)
-        ib = qkr.last_launch()
+        for pipe, u in [(1, 1), (1, 2), (1, 3), (1, 4), (3, 2)]:
+            qkr.tune_rope(pipe, u, 0, 0)
+            outs.append((run_fused(w, flags), qkr.last_launch()))
     finally:
-        qkr.tune_rope(0, 0, 0)
-    return a, b, ia, ib
+        qkr.tune_rope(0, 0, 0, 0)
+    return outs
 
 
-@pytest.mark.parametrize("case", ["joint-gptj", "joint-neox", "vit-d80", "partial-tile", "d256"])
-def test_pipelined_equals_register_kernel(case):
-    if case == "joint-gptj":
-        w = W.config3(seed=61, T_txt=77, img_h=9, img_w=13, H=24, D=128, pairing=W.PAIRING_GPTJ)
-    elif case == "joint-neox":
-        w = W.config3(seed=62, T_txt=64, img_h=8, img_w=8, H=24, D=128, pairing=W.PAIRING_NEOX)
-    elif case == "vit-d80":
-        pos = np.random.default_rng(3).integers(0, 4096, (1, 301)).astype(np.int32)
-        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=W.inv_freq(1e4, 32, 64).numpy())
-        w = W.random_rope_case(63, [301], 16, 16, 80, 64, W.PAIRING_NEOX, A)
-    elif case == "partial-tile":
-        pos = np.arange(7, dtype=np.int32)[None]
-        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=W.inv_freq(1e4, 32, 64).numpy())
-        w = W.random_rope_case(64, [7], 3, 1, 64, 64, W.PAIRING_GPTJ, A)
-    else:
-        pos = np.random.default_rng(4).integers(0, 9000, (1, 53)).astype(np.int32)
-        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=W.inv_freq(1e4, 128, 256).numpy())
-        w = W.random_rope_case(65, [53], 4, 2, 256, 256, W.PAIRING_NEOX, A)
-    (qa, ka), (qb, kb), ia, ib = _both_kernels(w)
-    assert ia["pipelined"] == 1 and ib["pipelined"] == 0
-    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
-    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+def _shape_cases():
+    cases = [("joint-gptj", W.config3(seed=61, T_txt=77, img_h=9, img_w=13, H=24, D=128,
+                                      pairing=W.PAIRING_GPTJ)),
+             ("joint-neox", W.config3(seed=62, T_txt=64, img_h=8, img_w=8, H=24, D=128,
+                                      pairing=W.PAIRING_NEOX))]
+    pos = np.random.default_rng(3).integers(0, 4096, (1, 301)).astype(np.int32)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 32, 64).numpy())
+    cases.append(("vit-d80", W.random_rope_case(63, [301], 16, 16, 80, 64, W.PAIRING_NEOX, A)))
+    pos = np.arange(7, dtype=np.int32)[None]
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 32, 64).numpy())
+    cases.append(("partial-tile", W.random_rope_case(64, [7], 3, 1, 64, 64, W.PAIRING_GPTJ, A)))
+    pos = np.random.default_rng(4).integers(0, 9000, (1, 53)).astype(np.int32)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 128, 256).numpy())
+    cases.append(("d256", W.random_rope_case(65, [53], 4, 2, 256, 256, W.PAIRING_NEOX, A)))
+    return cases
+
+
+@pytest.mark.parametrize("case,w", _shape_cases(), ids=lambda v: v if isinstance(v, str) else "")
+def test_heads_per_item_and_kernels_agree(case, w):
+    """Every heads-per-item choice of the item kernel and the streaming kernel
+    give the same bits, for both layouts, direct and staged angles and ragged
+    tiles, and match the oracle."""
+    outs = _shape_variants(w)
+    (q0, k0), _ = outs[0]
+    for (q, k), rec in outs[1:]:
+        assert torch.equal(q.view(torch.int16), q0.view(torch.int16)), (case, rec)
+        assert torch.equal(k.view(torch.int16), k0.view(torch.int16)), (case, rec)
+    assert outs[-1][1]["pipelined"] == 2 and outs[0][1]["pipelined"] == 0
     rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
-    assert_bf16_close(qa, rq, case + " q")
-    assert_bf16_close(ka, rk, case + " k")
+    assert_bf16_close(q0, rq, case + " q")
+    assert_bf16_close(k0, rk, case + " k")
 
 
-def test_pipelined_strided_heads_and_tile_sweep():
-    # non-dense head stride (one bulk copy per row) and every tile size
+def test_strided_heads_every_kernel_and_tile():
+    # non-dense head stride, both kernels, heads per item, ring depth and tile size
     g = torch.Generator().manual_seed(66)
     T, H, D = 41, 6, 128
     qkv = W.bf16_normal((T, H, 3, D), g)
@@ -268,20 +336,26 @@ def test_pipelined_strided_heads_and_tile_sweep():
     a = qkr.angle_positions(to_dev(pos), to_dev(inv))
     outs = []
     try:
-        for pipe, tt in [(1, 0), (2, 1), (2, 2), (2, 3), (2, 4)]:
-            qkr.tune_rope(pipe, 0, tt)
+        for pipe, u, tt, st in [(1, 0, 0, 0), (1, 2, 1, 0), (1, 4, 3, 0), (1, 1, 5, 0),
+                                (3, 2, 1, 2), (3, 4, 4, 3), (3, 1, 2, 4)]:
+            qkr.tune_rope(pipe, u, tt, st)
             qo = torch.empty(T, H, D, dtype=torch.bfloat16, device="cuda")
             ko = torch.empty_like(qo)
             qkr.fused_qk_norm_rope([(qv, kv, to_dev(gq), to_dev(gk))], qo, ko, D, W.PAIRING_NEOX,
                                    1e-6, a)
             torch.cuda.synchronize()
-            assert qkr.last_launch()["pipelined"] == (1 if pipe == 2 else 0)
+            assert qkr.last_launch()["pipelined"] == (2 if pipe == 3 else 0)
             outs.append((qo, ko))
     finally:
         qkr.tune_rope(0, 0, 0)
     for qo, ko in outs[1:]:
         assert torch.equal(qo.view(torch.int16), outs[0][0].view(torch.int16))
         assert torch.equal(ko.view(torch.int16), outs[0][1].view(torch.int16))
+    s = W.StreamInputs(qkv[:, :, 0].contiguous(), qkv[:, :, 1].contiguous(), gq, gk)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos, inv_freq=inv)
+    rq, rk = oracle.qk_norm_rope([s], H, H, D, D, W.PAIRING_NEOX, 1e-6, A)
+    assert_bf16_close(outs[0][0], rq, "strided heads q")
+    assert_bf16_close(outs[0][1], rk, "strided heads k")
 
 
 def _table_call(w, cos, sin, mode=W.SECTIONS_NONE, sections=None):

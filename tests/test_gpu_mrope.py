@@ -156,3 +156,26 @@ def test_gptj_sections_and_partial_rotary():
         rq, rk = oracle_mrope(w)
         assert_bf16_close(qo, rq, "partial q")
         assert_bf16_close(ko, rk, "partial k")
+
+
+def test_packed_qkv_in_place():
+    """Q and K rotated in place as column windows of one packed [T, 3, H, D]
+    buffer: their byte ranges interleave but share no element, so the call is
+    accepted, equals the fresh-output launch bit for bit and leaves V alone."""
+    w = W.config4(seed=91, T=300, Hq=8, Hkv=8)
+    q, k, pos, inv = _dev_inputs(w)
+    T, H, D = q.shape
+    g = torch.Generator(device="cuda").manual_seed(92)
+    buf = torch.empty(T, 3, H, D, dtype=torch.bfloat16, device="cuda")
+    buf[:, 0].copy_(q)
+    buf[:, 1].copy_(k)
+    buf[:, 2].copy_(torch.randn(T, H, D, device="cuda", generator=g).to(torch.bfloat16))
+    v_before = buf[:, 2].clone()
+    qv, kv = buf[:, 0], buf[:, 1]
+    qkr.mrope_apply(qv, kv, qv, kv, pos, inv, w.rot, w.angle.section_mode, w.angle.sections,
+                    w.pairing)
+    torch.cuda.synchronize()
+    ref_q, ref_k = run_mrope(w)
+    assert torch.equal(qv.view(torch.int16), ref_q.view(torch.int16))
+    assert torch.equal(kv.view(torch.int16), ref_k.view(torch.int16))
+    assert torch.equal(buf[:, 2].view(torch.int16), v_before.view(torch.int16))
