@@ -422,13 +422,16 @@ qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t token
  * last bit between choices; each choice is deterministic. */
 qkr_status qkr_tune_rope_lanes(int32_t lanes);
 
-/* CTAs that share one row in rms_norm_residual / rms_norm_fp8, for tuning
- * sweeps: 0 automatic (a cluster of 8 or 4 CTAs for up to 32 rows, else one
- * CTA per row), else 1, 2, 4, 8 or 16 (a thread-block cluster when > 1).
- * Process-wide.  The split sets the order of the fp32 sum of squares, so the
- * normalised output can differ in the last bit between choices; the residual
- * stream is bit-identical. */
-qkr_status qkr_tune_rms(int32_t cluster);
+/* CTAs that share one row in rms_norm_residual / rms_norm_fp8, and the
+ * threads of each CTA, for tuning sweeps.  cluster: 0 automatic, else 1, 2,
+ * 4, 8 or 16 (a thread-block cluster when > 1).  threads: 0 automatic, else a
+ * multiple of 32 in [32, 1024]: the CTA width the row slice is spread over
+ * (each thread keeps its 16-byte vectors of the slice in registers, so a
+ * wider CTA holds fewer per thread).  Process-wide.  The split and the width
+ * set the order of the fp32 sum of squares, so the normalised output can
+ * differ in the last bit between choices; the residual stream is
+ * bit-identical. */
+qkr_status qkr_tune_rms(int32_t cluster, int32_t threads);
 
 /* Device status word of the library on the current device (0 = healthy).
  * Bit 4: rope_set_rows met a row index outside the cache (that row was not

@@ -94,7 +94,7 @@ def _load() -> ctypes.CDLL:
         "qkr_vit_positions": [V, V, V, I64, I64, I64, V],
         "qkr_tune_rope": [I32, I32, I32, I32],
         "qkr_tune_rope_lanes": [I32],
-        "qkr_tune_rms": [I32],
+        "qkr_tune_rms": [I32, I32],
         "qkr_launch_overlap": [I32],
         "qkr_device_status": [ctypes.POINTER(ctypes.c_uint32), I32],
         "qkr_null_launch": [V, I64, I32],
@@ -175,9 +175,10 @@ def tune_rope_lanes(lanes: int = 0) -> None:
     _check(_lib.qkr_tune_rope_lanes(lanes))
 
 
-def tune_rms(cluster: int = 0) -> None:
-    """CTAs per row of the RMSNorm kernels (0 = automatic), for tuning."""
-    _check(_lib.qkr_tune_rms(cluster))
+def tune_rms(cluster: int = 0, threads: int = 0) -> None:
+    """CTAs per row and threads per CTA of the RMSNorm kernels (0 = automatic),
+    for tuning."""
+    _check(_lib.qkr_tune_rms(cluster, threads))
 
 
 def launch_overlap(enable: bool) -> None:

@@ -481,12 +481,14 @@ qkr_status qkr_launch_overlap(int32_t enable)
     return QKR_OK;
 }
 
-qkr_status qkr_tune_rms(int32_t cluster)
+qkr_status qkr_tune_rms(int32_t cluster, int32_t threads)
 {
     if (cluster != 0 && cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8 &&
         cluster != 16)
         return fail(QKR_ERR_INVALID_ARG, "cluster must be 0 or a power of two up to 16");
-    qkr::set_rms_cluster_override(cluster);
+    if (threads != 0 && (threads < 32 || threads > 1024 || threads % 32))
+        return fail(QKR_ERR_INVALID_ARG, "threads must be 0 or a multiple of 32 in [32, 1024]");
+    qkr::set_rms_cluster_override(cluster, threads);
     g_error.clear();
     return QKR_OK;
 }

@@ -241,7 +241,7 @@ struct RmsParams {
 };
 cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream,
                                      LaunchRecord *rec);
-// CTAs per row of the RMSNorm kernels, for tuning (0: automatic).
-void set_rms_cluster_override(int cluster);
+// CTAs per row and threads per CTA of the RMSNorm kernels, for tuning (0: automatic).
+void set_rms_cluster_override(int cluster, int threads);
 
 }  // namespace qkr

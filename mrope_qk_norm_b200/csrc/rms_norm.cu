@@ -201,6 +201,7 @@ Fn cluster_fn(int vpt)
 }
 
 std::atomic<int> g_force_cluster{0};  // tuning override of CTAs per row (0: automatic)
+std::atomic<int> g_force_threads{0};  // tuning override of threads per CTA (0: automatic)
 
 // Smallest power-of-two vectors-per-thread keeping the block at or under
 // `target` threads (and never above 1024).
@@ -217,7 +218,11 @@ void shape(int vectors, int target, int &vpt, int &threads)
 
 }  // namespace
 
-void set_rms_cluster_override(int cluster) { g_force_cluster = cluster; }
+void set_rms_cluster_override(int cluster, int threads)
+{
+    g_force_cluster = cluster;
+    g_force_threads = threads;
+}
 
 cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, LaunchRecord *rec)
 {
@@ -236,7 +241,8 @@ cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, La
         cs = g_force_cluster;
     int vpt, threads;
     const int per = (nvec + cs - 1) / cs;
-    shape(per, 256, vpt, threads);
+    const int target = g_force_threads > 0 ? (int)g_force_threads : 256;
+    shape(per, target, vpt, threads);
     if ((int64_t)threads * vpt < per)
         return cudaErrorInvalidConfiguration;
     const int64_t grid = p.R * cs;

@@ -95,6 +95,28 @@ def test_setup_many_grids_and_long_axis():
     assert np.array_equal(cos.untouched(), ~mask)
 
 
+@pytest.mark.parametrize("lens,m", [((64, 64, 64), 1), ((4, 6, 6), 1), ((16, 24, 24), 4)])
+def test_setup_empty_grids_and_narrow_grids(lens, m):
+    """Grids with zero frames among at most 32 grids (the kernel finds a
+    token's grid by shuffles over the boundaries), merge sizes 1 and 4, and
+    grids one merge block wide (8 consecutive tokens of a warp then span 8
+    h positions): planes and positions equal the oracle's."""
+    grids = [[1, 8 * m, m], [0, 4 * m, 4 * m], [2, 2 * m, 6 * m], [0, m, m], [1, 16 * m, m],
+             [1, 4 * m, 4 * m]]
+    w = W.config5(seed=57, grids=grids, lens=lens, spatial_merge=m)
+    cos, sin, cu, dgrids, N = run_setup(w)
+    pos = oracle.vit_positions(w.grids, m)
+    rc, rs, written = oracle.vit_planes(pos, w.inv_t, w.inv_h, w.inv_w)
+    mask = written.astype(bool)
+    assert_plane_close(cos.tensor.cpu().numpy(), rc, mask, "cos")
+    assert_plane_close(sin.tensor.cpu().numpy(), rs, mask, "sin")
+    assert np.array_equal(cos.untouched(), ~mask)
+    out = torch.empty(3, N, dtype=torch.int32, device="cuda")
+    qkr.vit_positions(cu, dgrids, N, m, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), pos)
+
+
 def test_setup_empty_grid_list():
     inv = torch.ones(4, dtype=torch.float32, device="cuda")
     e32 = torch.empty(0, dtype=torch.int32, device="cuda")
