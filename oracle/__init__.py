@@ -25,6 +25,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 SEC_NONE, SEC_CONTIGUOUS, SEC_INTERLEAVED, SEC_INTERLEAVED_QUOTA, SEC_IMROPE = range(5)
+# Rounding points of the normalised value (oracle.c rms_norm_head).
+ROUND_NONE, ROUND_NORMALIZED, ROUND_EAGER = range(3)
 
 
 def build(force: bool = False) -> str:
@@ -61,7 +63,7 @@ def _load():
         lib.oracle_qk_norm_rope.restype = I32
         lib.oracle_qk_norm_rope.argtypes = [I32, P, P, P, P, P, I64, I64, I64, I64, I32,
                                             ctypes.c_double, I32, I32,
-                                            ctypes.POINTER(_Angle), P, P]
+                                            ctypes.POINTER(_Angle), P, P, P, P]
         lib.oracle_vit_positions.restype = I64
         lib.oracle_vit_positions.argtypes = [P, I64, ctypes.c_int32, P, I64]
         lib.oracle_vit_planes.restype = None
@@ -145,12 +147,21 @@ def _make_angle(angle, keep: list) -> _Angle:
 
 
 def qk_norm_rope(streams, Hq: int, Hk: int, D: int, rot: int, pairing: int, eps: float,
-                 angle, norm: bool = True, round_normalized: bool = False):
+                 angle, norm: bool = True, round_normalized: bool = False,
+                 eager_rounding: bool = False, return_ties: bool = False):
     """Joint (text-first) RMSNorm + RoPE of Q and K; returns fp64 [T, H, D] arrays.
 
     ``streams`` is a list of objects with ``q``, ``k`` ([T, H, D] bf16) and
-    ``gamma_q``, ``gamma_k`` ([D] bf16) attributes.
+    ``gamma_q``, ``gamma_k`` ([D] bf16) attributes.  ``round_normalized``:
+    y = bf16(x r gamma) before the rotation; ``eager_rounding``: y =
+    bf16(bf16(x r) gamma).  With ``return_ties`` also returns two uint8 masks
+    of the output elements that depend on a value sitting within 1e-3 bf16
+    quanta of a rounding midpoint (where an fp32 evaluation may take the
+    other neighbour).
     """
+    if round_normalized and eager_rounding:
+        raise ValueError("one rounding contract at a time")
+    mode = ROUND_EAGER if eager_rounding else (ROUND_NORMALIZED if round_normalized else ROUND_NONE)
     lib = _load()
     keep = []
     T_s = np.array([int(s.q.shape[0]) for s in streams], dtype=np.int64)
@@ -162,17 +173,22 @@ def qk_norm_rope(streams, Hq: int, Hk: int, D: int, rot: int, pairing: int, eps:
     T = int(T_s.sum())
     q_out = np.empty((T, Hq, D), dtype=np.float64)
     k_out = np.empty((T, Hk, D), dtype=np.float64)
+    tq = np.zeros((T, Hq, D), dtype=np.uint8) if return_ties else None
+    tk = np.zeros((T, Hk, D), dtype=np.uint8) if return_ties else None
     A = _make_angle(angle, keep)
     rc = lib.oracle_qk_norm_rope(len(streams), _ptr(T_s),
                                  ctypes.cast(ptrs["q"], ctypes.c_void_p),
                                  ctypes.cast(ptrs["k"], ctypes.c_void_p),
                                  ctypes.cast(ptrs["gamma_q"], ctypes.c_void_p),
                                  ctypes.cast(ptrs["gamma_k"], ctypes.c_void_p),
-                                 Hq, Hk, D, rot, pairing, float(eps), int(norm),
-                                 int(round_normalized), ctypes.byref(A),
-                                 _ptr(q_out), _ptr(k_out))
+                                 Hq, Hk, D, rot, pairing, float(eps), int(norm), mode,
+                                 ctypes.byref(A), _ptr(q_out), _ptr(k_out),
+                                 _ptr(tq) if return_ties else None,
+                                 _ptr(tk) if return_ties else None)
     if rc != 0:
         raise ValueError("oracle_qk_norm_rope rejected its arguments")
+    if return_ties:
+        return q_out, k_out, tq.astype(bool), tk.astype(bool)
     return q_out, k_out
 
 

@@ -15,8 +15,11 @@
  *     (vllm.cpp #185 "decode RmsNorm ran on ONE workgroup", the
  *     vt_round_through paragraph: the summed residual carries bf16 rounding);
  *   - optionally, the normalised value is rounded to bf16 before rotation
- *     (vllm-omni #7600, review of the interleaved tile: "bf16-rounded
- *     normalized value, fp32 rotation, one final rounding").
+ *     (vllm-omni #7600, review of the interleaved tile: a bf16-rounded
+ *     normalised value, an fp32 rotation and one final rounding), or rounded
+ *     at the two points of the eager RMSNorm (vLLM #26234, rms_norm_kernel:
+ *     the normalised value cast to bf16, then a bf16 product with the
+ *     weight).
  * Outputs are returned unrounded (fp64), except bf16 streams that are
  * themselves the result (the residual) and fp32 planes.
  *
@@ -192,9 +195,42 @@ static void angle_of(const oracle_angle *A, int64_t n, int64_t j, double *c, dou
 
 /* ----------------------------------------------------- per-row helpers -- */
 
-/* y = x / sqrt(mean(x^2) + eps) * gamma  (RMSNorm over the head dim). */
+/* Rounding points of the normalised value (see oracle_qk_norm_rope). */
+enum { ROUND_NONE = 0, ROUND_NORMALIZED = 1, ROUND_EAGER = 2 };
+
+/* Distance, in bf16 quanta, below which a value counts as sitting on a
+ * rounding midpoint: a single-precision evaluation of the same value (the
+ * GPU's fp32 sum of squares and rsqrt differ from fp64 by about 1e-6
+ * relative, a few 1e-4 quanta) may round it to the other neighbour. */
+#define TIE_TOL 1e-3
+
+/* 1 if v lies within TIE_TOL quanta of a bf16 rounding midpoint. */
+static int near_bf16_tie(double v)
+{
+    double a = fabs(v);
+    if (a == 0.0 || isinf(a) || isnan(a))
+        return 0;
+    int ex;
+    frexp(a, &ex);
+    int quantum = ex - 8;
+    if (quantum < -133)
+        quantum = -133;
+    double u = ldexp(a, -quantum);   /* a in quanta */
+    double f = u - floor(u);
+    return fabs(f - 0.5) < TIE_TOL;
+}
+
+/* y = x / sqrt(mean(x^2) + eps) * gamma  (RMSNorm over the head dim), with the
+ * rounding points of round_mode:
+ *   ROUND_NONE        y unrounded;
+ *   ROUND_NORMALIZED  y = bf16(x r gamma);
+ *   ROUND_EAGER       y = bf16(bf16(x r) * gamma): the eager RMSNorm casts the
+ *                     normalised value to the activation type, then multiplies
+ *                     it by the bf16 weight with a bf16 result (vLLM #26234,
+ *                     the rms_norm_kernel line the review quotes).
+ * tie[d] (nullable) = 1 where the value rounded first sat on a midpoint. */
 static void rms_norm_head(const uint16_t *x, const uint16_t *gamma, int64_t D, double eps,
-                          double *y)
+                          int round_mode, double *y, uint8_t *tie)
 {
     double ss = 0.0;
     for (int64_t d = 0; d < D; ++d) {
@@ -202,8 +238,23 @@ static void rms_norm_head(const uint16_t *x, const uint16_t *gamma, int64_t D, d
         ss += v * v;
     }
     double inv_rms = 1.0 / sqrt(ss / (double)D + eps);
-    for (int64_t d = 0; d < D; ++d)
-        y[d] = bf16_value(x[d]) * inv_rms * bf16_value(gamma[d]);
+    for (int64_t d = 0; d < D; ++d) {
+        double xr = bf16_value(x[d]) * inv_rms;
+        double g = bf16_value(gamma[d]);
+        if (round_mode == ROUND_EAGER) {
+            if (tie)
+                tie[d] = (uint8_t)near_bf16_tie(xr);
+            y[d] = bf16_rounded_value(bf16_rounded_value(xr) * g);
+        } else if (round_mode == ROUND_NORMALIZED) {
+            if (tie)
+                tie[d] = (uint8_t)near_bf16_tie(xr * g);
+            y[d] = bf16_rounded_value(xr * g);
+        } else {
+            if (tie)
+                tie[d] = 0;
+            y[d] = xr * g;
+        }
+    }
 }
 
 /* Rotate the first rot dims in pairs: NeoX pairs (j, j + rot/2), GPT-J pairs
@@ -228,17 +279,27 @@ static void rotate_head(double *y, int64_t rot, int pairing, const oracle_angle 
  * Streams are dense [T_s, H, D] bf16 (bits).  The joint output is the
  * concatenation over streams in order (text first), [sum T_s, H, D], fp64.
  * do_norm = 0 skips the RMSNorm (plain rotation of the input values).
+ * round_mode (with do_norm): the rounding points of the normalised value, as
+ * rms_norm_head states them; the rotation itself is exact (fp64) and the
+ * output unrounded.
+ * tie_q / tie_k (nullable, [sum T_s, H, D]): 1 where an output element
+ * depends on a normalised value that sat on a bf16 rounding midpoint (the
+ * element itself, or its rotation partner).
  */
 int oracle_qk_norm_rope(int n_streams, const int64_t *T_s,
                         const uint16_t *const *q_s, const uint16_t *const *k_s,
                         const uint16_t *const *gq_s, const uint16_t *const *gk_s,
                         int64_t Hq, int64_t Hk, int64_t D, int64_t rot, int pairing,
-                        double eps, int do_norm, int round_normalized,
-                        const oracle_angle *A, double *q_out, double *k_out)
+                        double eps, int do_norm, int round_mode,
+                        const oracle_angle *A, double *q_out, double *k_out,
+                        uint8_t *tie_q, uint8_t *tie_k)
 {
     if (D <= 0 || rot < 0 || rot > D || (rot & 1) || D > 4096)
         return -1;
+    if (round_mode < ROUND_NONE || round_mode > ROUND_EAGER)
+        return -1;
     double y[4096];
+    uint8_t tie[4096];
     int64_t n = 0;                  /* joint token index */
     for (int s = 0; s < n_streams; ++s) {
         for (int64_t t = 0; t < T_s[s]; ++t, ++n) {
@@ -247,18 +308,30 @@ int oracle_qk_norm_rope(int n_streams, const int64_t *T_s,
                 const uint16_t *src = which == 0 ? q_s[s] : k_s[s];
                 const uint16_t *gam = which == 0 ? gq_s[s] : gk_s[s];
                 double *dst = which == 0 ? q_out : k_out;
+                uint8_t *tdst = which == 0 ? tie_q : tie_k;
                 for (int64_t h = 0; h < H; ++h) {
                     const uint16_t *x = src + (t * H + h) * D;
-                    if (do_norm)
-                        rms_norm_head(x, gam, D, eps, y);
-                    else
-                        for (int64_t d = 0; d < D; ++d)
+                    if (do_norm) {
+                        rms_norm_head(x, gam, D, eps, round_mode, y, tie);
+                    } else {
+                        for (int64_t d = 0; d < D; ++d) {
                             y[d] = bf16_value(x[d]);
-                    if (round_normalized)
-                        for (int64_t d = 0; d < D; ++d)
-                            y[d] = bf16_rounded_value(y[d]);
+                            tie[d] = 0;
+                        }
+                    }
                     rotate_head(y, rot, pairing, A, n);
                     memcpy(dst + (n * H + h) * D, y, (size_t)D * sizeof(double));
+                    if (tdst) {
+                        uint8_t *to = tdst + (n * H + h) * D;
+                        memcpy(to, tie, (size_t)D);
+                        for (int64_t j = 0; j < rot / 2; ++j) {
+                            int64_t ia = pairing == 0 ? j : 2 * j;
+                            int64_t ib = pairing == 0 ? j + rot / 2 : 2 * j + 1;
+                            uint8_t any = (uint8_t)(tie[ia] | tie[ib]);
+                            to[ia] = any;
+                            to[ib] = any;
+                        }
+                    }
                 }
             }
         }

@@ -412,6 +412,89 @@ def test_round_normalized_contract():
     assert np.array_equal(rnd, lib)
 
 
+def _eager_case():
+    x = _bf16([1, 1, 7, 1, 1, 1, 1, 1]).reshape(1, 1, 8)
+    g = _bf16([1.5, 0.75, 1, 1, 1, 1, 1, 1])
+    return _S(x, x, g, g)
+
+
+@pytest.mark.parametrize("contract", ["eager", "round_normalized", "none"])
+def test_rounding_contracts_hand_worked(contract):
+    """The three rounding contracts on the hand-worked row of
+    tests/golden/eager_rounding.txt, at position 0 (identity rotation)."""
+    rows = {}
+    with open(os.path.join(GOLDEN, "eager_rounding.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, ys = [p.strip() for p in line.split("|")]
+            rows[name] = [float(v) for v in ys.split()]
+    q, _ = oracle.qk_norm_rope([_eager_case()], 1, 1, 8, 8, W.PAIRING_GPTJ, 0.0,
+                               _pos_angle([0], np.zeros(4)),
+                               round_normalized=contract == "round_normalized",
+                               eager_rounding=contract == "eager")
+    np.testing.assert_allclose(q.reshape(-1), rows[contract], rtol=1e-15, atol=0)
+    if contract != "none":
+        assert rows["eager"][:2] != rows["round_normalized"][:2]  # the example separates them
+
+
+def test_eager_rounding_happens_before_the_rotation():
+    """With a table angle (cos, sin) = (fp32 0.6, fp32 0.8) on every pair, the
+    eager output is the textbook rotation of the hand-worked rounded values
+    (rounding first, then the exact rotation, no rounding after it)."""
+    c, s = float(np.float32(0.6)), float(np.float32(0.8))
+    cos = np.full((1, 4), c, dtype=np.float32)
+    sin = np.full((1, 4), s, dtype=np.float32)
+    A = W.AngleInputs(kind=W.ANGLE_TABLE, cos=cos, sin=sin)
+    q, _ = oracle.qk_norm_rope([_eager_case()], 1, 1, 8, 8, W.PAIRING_GPTJ, 0.0, A,
+                               eager_rounding=True)
+    y = [0.5703125, 0.28515625, 2.640625] + [0.37890625] * 5
+    want = []
+    for j in range(4):
+        a, b = y[2 * j], y[2 * j + 1]
+        want += [a * c - b * s, b * c + a * s]
+    np.testing.assert_allclose(q.reshape(-1), want, rtol=1e-15, atol=1e-15)
+
+
+def test_eager_rounding_is_two_roundings_of_torch():
+    """On random rows the eager contract equals torch's bf16 rounding (RNE, a
+    library pin) applied to x r and then to the rounded value times gamma,
+    with r from the unrounded contract's own output (y = x r gamma)."""
+    g = torch.Generator().manual_seed(12)
+    T, H, D = 4, 3, 64
+    x = W.bf16_normal((T, H, D), g)
+    gam = W.bf16_uniform((D,), 0.5, 1.5, g)
+    A = _pos_angle(np.zeros(T), W.inv_freq(1e4, 32, 64).numpy())
+    exact = oracle.qk_norm_rope([_S(x, x, gam, gam)], H, H, D, D, 0, 1e-6, A)[0]
+    eager = oracle.qk_norm_rope([_S(x, x, gam, gam)], H, H, D, D, 0, 1e-6, A,
+                                eager_rounding=True)[0]
+    xr = exact / _f64(gam)                       # x r per element
+    n = torch.from_numpy(xr).to(torch.bfloat16).double()
+    want = (n * torch.from_numpy(_f64(gam))).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(eager, want)
+    assert not np.array_equal(eager, exact)
+
+
+def test_tie_masks():
+    """The near-tie masks: empty without intermediate rounding, shared by both
+    members of every rotation pair, and about 2e-3 of the elements (values
+    within 1e-3 quanta of a midpoint) on random rows."""
+    g = torch.Generator().manual_seed(13)
+    T, H, D = 64, 8, 128
+    x = W.bf16_normal((T, H, D), g)
+    gam = W.bf16_uniform((D,), 0.5, 1.5, g)
+    A = _pos_angle(np.arange(T), W.inv_freq(1e4, 64, 128).numpy())
+    _, _, tq0, _ = oracle.qk_norm_rope([_S(x, x, gam, gam)], H, H, D, D, 0, 1e-6, A,
+                                       return_ties=True)
+    assert not tq0.any()
+    for kw in ({"eager_rounding": True}, {"round_normalized": True}):
+        _, _, tq, tk = oracle.qk_norm_rope([_S(x, x, gam, gam)], H, H, D, D, 0, 1e-6, A,
+                                           return_ties=True, **kw)
+        assert np.array_equal(tq[..., :64], tq[..., 64:])     # NeoX pairs (j, j + 64)
+        frac = tq.mean()
+        assert 5e-4 < frac < 1.2e-2, frac
+
+
 # ------------------------------------------------------------ ViT setup --
 
 def _unravel_positions(grids, m):
