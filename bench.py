@@ -307,17 +307,23 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
         s4.append((q, k, torch.empty_like(q), torch.empty_like(k)))
     pos4, inv4 = w4.angle.positions.to(dev), w4.angle.inv_freq.to(dev)
 
-    def mr(x, chunks):
+    def mr(x, chunks, independent=False):
         q, k, qo_, ko_ = x
-        for t0, t1 in chunks:
+        for i, (t0, t1) in enumerate(chunks):
+            # QKR_FLAG_INDEPENDENT: a later chunk of the step touches nothing
+            # the earlier chunk does
             qkr.mrope_apply(q[t0:t1], k[t0:t1], qo_[t0:t1], ko_[t0:t1], pos4, inv4, 128,
                             W.SECTIONS_INTERLEAVED, (24, 20, 20), 0, token_offset=t0,
+                            flags=qkr.FLAG_INDEPENDENT if independent and i else 0,
                             stream=stream)
     record("mrope_apply", "interleaved mRoPE T=8192 Hq=16 Hkv=8 D=128 (24,20,20)",
            [lambda x=x: mr(x, [(0, 8192)]) for x in s4], b4, 8192, "tokens")
     record("mrope_apply", "same, two chunked launches split at 2457 (per step)",
            [lambda x=x: mr(x, [(0, 2457), (2457, 8192)]) for x in s4], b4, 8192, "tokens",
            {"launches_per_step": 2})
+    record("mrope_apply", "same, chunked at 2457, second chunk flagged independent (per step)",
+           [lambda x=x: mr(x, [(0, 2457), (2457, 8192)], True) for x in s4], b4, 8192,
+           "tokens", {"launches_per_step": 2, "flags": "QKR_FLAG_INDEPENDENT on chunk 2"})
     del s4
 
     # rope + set_rows: config 4's K rows rotated and scattered into a 16384-row cache
@@ -461,7 +467,7 @@ def _oracle_sample():
     return step, tokens
 
 
-def cpu_baseline(budget_s: float = 12.0) -> dict:
+def cpu_baseline(budget_s: float = 8.0) -> dict:
     """The oracle as it stands, single-threaded, on a bounded token sample."""
     step, tokens = _oracle_sample()
     t0 = time.perf_counter()
@@ -479,7 +485,7 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
                       % (calls, tokens, N_IMG_SAMPLE, dt)}
 
 
-def cpu_baseline_parallel(budget_s: float = 8.0) -> dict:
+def cpu_baseline_parallel(budget_s: float = 5.0) -> dict:
     """The same oracle run concurrently on every host core the process may use:
     thread i repeatedly processes its own slice of the image stream (the
     oracle is C called through ctypes, which releases the GIL)."""
@@ -517,6 +523,321 @@ def cpu_baseline_parallel(budget_s: float = 8.0) -> dict:
     return {"value": round(total / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": "%d threads, each repeating the oracle on its own %d-token slice of the "
                       "headline's image stream, %.1f s" % (cores, per, dt)}
+
+
+# ------------------------------------------- per-row oracle legs (CPU) --
+#
+# For every row: the oracle timed on a bounded sample of that row's own
+# workload (one thread, then every host core), and the GPU output of the same
+# launch shape as the timed one compared with the oracle on that sample.  The
+# oracle runs on the CPU only; the GPU outputs come from a separate launch on
+# fresh inputs (the timed launches rotate over copies and rewrite residuals).
+
+LEG_SAMPLE = 1024      # tokens (rope rows) in a sample
+LEG_ROWS = 256         # rows (RMSNorm rows) in a sample
+LEG_BUDGET_S = 0.4     # seconds of oracle time per leg and per mode
+
+
+def _err_report(got: np.ndarray, ref: np.ndarray, what: str) -> dict:
+    err = np.abs(got - ref)
+    bound = 1e-2 + 1.6e-2 * np.abs(ref)
+    den = float((ref ** 2).sum())
+    return {"elements": int(ref.size), "max_abs": float(err.max()) if err.size else 0.0,
+            "nmse": float(((got - ref) ** 2).sum()) / den if den > 0 else 0.0,
+            "outside_tolerance": int((~(err <= bound)).sum()), "sample": what}
+
+
+def _time_leg(run, units: int, slices, unit: str, sample: str) -> tuple:
+    """(single-thread, all-cores) oracle throughput: run() processes `units`;
+    slices is a list of (callable, units) covering the sample for the
+    parallel leg (the oracle is C through ctypes, which releases the GIL)."""
+    import concurrent.futures
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        run()
+        n += 1
+        if time.perf_counter() - t0 >= LEG_BUDGET_S:
+            break
+    dt = time.perf_counter() - t0
+    single = {"value": round(n * units / dt, 1), "unit": unit + "/s", "cores": 1,
+              "kind": "oracle", "sample": sample + "; %d calls in %.2f s" % (n, dt)}
+    cores = max(1, min(len(os.sched_getaffinity(0)), 64, len(slices)))
+    t_end = time.perf_counter() + LEG_BUDGET_S
+
+    def work(i):
+        fn, u = slices[i % len(slices)]
+        done = 0
+        while time.perf_counter() < t_end:
+            fn()
+            done += u
+        return done
+
+    t1 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=cores) as ex:
+        total = sum(ex.map(work, range(cores)))
+    dt1 = time.perf_counter() - t1
+    allc = {"value": round(total / dt1, 1), "unit": unit + "/s", "cores": cores,
+            "kind": "oracle", "sample": sample + "; %d threads, one slice each" % cores}
+    return single, allc
+
+
+def _token_slices(make, n_units: int, parts: int):
+    """Split a sample of n_units tokens (rows) into at most `parts` oracle
+    calls of at least 16 units each (one per host thread: smaller calls are
+    bound by the Python side of the call, which holds the interpreter lock)."""
+    parts = max(1, min(parts, len(os.sched_getaffinity(0)), n_units // 16))
+    per = max(1, -(-n_units // parts))
+    out = []
+    for a in range(0, n_units, per):
+        b = min(n_units, a + per)
+        out.append((make(a, b), b - a))
+    return out
+
+
+def _leg_rope(w, out_q, out_k, rows, sub_streams, angle_for, sample, **kw):
+    """A rope row: out_q/out_k are the GPU's joint outputs (host bf16
+    tensors); rows = the joint rows the sample covers; sub_streams(a, b) the
+    oracle's streams for sample tokens [a, b); angle_for(a) its angle input."""
+    import oracle
+    n = len(rows)
+
+    def run_range(a, b):
+        return oracle.qk_norm_rope(sub_streams(a, b), w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps,
+                                   angle_for(a), norm=w.norm, **kw)
+    rq, rk = run_range(0, n)
+    g = np.concatenate([out_q[rows].float().numpy().astype(np.float64).reshape(-1),
+                        out_k[rows].float().numpy().astype(np.float64).reshape(-1)])
+    err = _err_report(g, np.concatenate([rq.reshape(-1), rk.reshape(-1)]), sample)
+    single, allc = _time_leg(lambda: run_range(0, n), n,
+                             _token_slices(lambda a, b: (lambda: run_range(a, b)), n, 64),
+                             "tokens", sample)
+    return {"cpu_baseline": single, "cpu_baseline_all_cores": allc, "error_vs_oracle": err}
+
+
+def oracle_legs(dev, stream) -> dict:
+    """Per-row CPU baselines and GPU-vs-oracle errors, keyed by row workload."""
+    import mrope_qk_norm_b200 as qkr
+    import oracle
+    legs = {}
+    S = LEG_SAMPLE
+
+    def joint_sub(w):
+        txt, img = w.streams
+        T_txt = txt.q.shape[0]
+
+        def sub(a, b):
+            # sample tokens [a, b) of [all text, first S - T_txt image tokens]
+            out = []
+            if a < T_txt:
+                out.append(W.StreamInputs(txt.q[a:min(b, T_txt)], txt.k[a:min(b, T_txt)],
+                                          txt.gamma_q, txt.gamma_k))
+            ia, ib = max(a, T_txt) - T_txt, b - T_txt
+            if ib > ia:
+                out.append(W.StreamInputs(img.q[ia:ib], img.k[ia:ib], img.gamma_q, img.gamma_k))
+            return out
+        return sub
+
+    def table_at(w):
+        return lambda a: W.AngleInputs(kind=w.angle.kind, cos=w.angle.cos, sin=w.angle.sin,
+                                       token_offset=a)
+
+    # config 1
+    w = W.config1()
+    s0 = w.streams[0]
+    d = [t.to(dev) for t in (s0.q, s0.k, s0.gamma_q, s0.gamma_k)]
+    qo, ko = torch.empty_like(d[0]), torch.empty_like(d[1])
+    qkr.fused_qk_norm_rope([tuple(d)], qo, ko, w.rot, w.pairing, w.eps,
+                           qkr.angle_positions(w.angle.positions.to(dev),
+                                               w.angle.inv_freq.to(dev)), 0, stream)
+    torch.cuda.synchronize()
+    T1 = s0.q.shape[0]
+    legs["single-stream T=16 H=4 D=64 NeoX"] = _leg_rope(
+        w, qo.cpu(), ko.cpu(), list(range(T1)),
+        lambda a, b: [W.StreamInputs(s0.q[a:b], s0.k[a:b], s0.gamma_q, s0.gamma_k)],
+        lambda a: W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=w.angle.positions,
+                                inv_freq=w.angle.inv_freq, token_offset=a),
+        "all 16 tokens")
+
+    # config 3, both pairings (the GPT-J one is the headline), and Q/K/V
+    for pairing, key in ((W.PAIRING_GPTJ, "headline"),
+                         (W.PAIRING_NEOX, "joint 512+4096 tokens H=24 D=128 NeoX")):
+        w = W.config3(pairing=pairing)
+        fs = FusedSet(w, dev)
+        fs.launch(stream)
+        torch.cuda.synchronize()
+        legs[key] = _leg_rope(w, fs.qo.cpu(), fs.ko.cpu(), list(range(S)), joint_sub(w),
+                              table_at(w), "joint rows 0..%d (all 512 text + the first %d "
+                              "image tokens)" % (S - 1, S - 512))
+        if pairing == W.PAIRING_GPTJ:
+            g = torch.Generator(device=dev)
+            g.manual_seed(3000)
+            vs = [torch.randn(t[0].shape, device=dev, generator=g).to(torch.bfloat16)
+                  for t in fs.streams]
+            descs = [qkr.stream_desc(t[0], t[1], t[2], t[3], v) for t, v in zip(fs.streams, vs)]
+            vo = torch.empty(w.n_tokens, 24, 128, dtype=torch.bfloat16, device=dev)
+            qkr.fused_qkv_norm_rope(descs, fs.qo, fs.ko, vo, 128, w.pairing, w.eps, fs.angle, 0,
+                                    stream)
+            torch.cuda.synchronize()
+            leg = _leg_rope(w, fs.qo.cpu(), fs.ko.cpu(), list(range(S)), joint_sub(w),
+                            table_at(w), "joint rows 0..%d; V: every row" % (S - 1))
+            vref = oracle.joint_v([v.cpu() for v in vs])
+            leg["error_vs_oracle"]["v_rows_bit_exact"] = bool(
+                np.array_equal(oracle.bits(vo.cpu()), vref))
+            legs["joint Q/K/V 512+4096 tokens H=24 D=128 GPT-J"] = leg
+        del fs
+
+    # config 4: interleaved mRoPE, whole and chunked
+    w4 = W.config4()
+    s4 = w4.streams[0]
+    q, k = s4.q.to(dev), s4.k.to(dev)
+    pos4, inv4 = w4.angle.positions.to(dev), w4.angle.inv_freq.to(dev)
+
+    def mr(chunks):
+        qo_, ko_ = torch.empty_like(q), torch.empty_like(k)
+        for t0, t1 in chunks:
+            qkr.mrope_apply(q[t0:t1], k[t0:t1], qo_[t0:t1], ko_[t0:t1], pos4, inv4, 128,
+                            W.SECTIONS_INTERLEAVED, (24, 20, 20), 0, token_offset=t0,
+                            stream=stream)
+        torch.cuda.synchronize()
+        return qo_.cpu(), ko_.cpu()
+
+    def pos_at(a):
+        return W.AngleInputs(kind=W.ANGLE_POSITIONS, section_mode=w4.angle.section_mode,
+                             sections=w4.angle.sections, positions=w4.angle.positions,
+                             inv_freq=w4.angle.inv_freq, token_offset=a)
+    qo4, ko4 = mr([(0, 8192)])
+    legs["interleaved mRoPE T=8192 Hq=16 Hkv=8 D=128 (24,20,20)"] = _leg_rope(
+        w4, qo4, ko4, list(range(S)),
+        lambda a, b: [W.StreamInputs(s4.q[a:b], s4.k[a:b], s4.gamma_q, s4.gamma_k)],
+        pos_at, "tokens 0..%d" % (S - 1))
+    qc, kc = mr([(0, 2457), (2457, 8192)])
+    c0 = 2457
+    leg = _leg_rope(w4, qc, kc, list(range(c0, c0 + S)),
+                    lambda a, b: [W.StreamInputs(s4.q[c0 + a:c0 + b], s4.k[c0 + a:c0 + b],
+                                                 s4.gamma_q, s4.gamma_k)],
+                    lambda a: pos_at(c0 + a),
+                    "tokens %d..%d (the second chunk's first %d)" % (c0, c0 + S - 1, S))
+    leg["error_vs_oracle"]["chunked_equals_whole_bit_exact"] = bool(
+        torch.equal(qc.view(torch.int16), qo4.view(torch.int16)) and
+        torch.equal(kc.view(torch.int16), ko4.view(torch.int16)))
+    legs["same, two chunked launches split at 2457 (per step)"] = leg
+
+    # rope_set_rows
+    g_sr = torch.Generator(device=dev)
+    g_sr.manual_seed(4100)
+    cache = torch.full((16384, 8, 128), float("nan"), dtype=torch.bfloat16, device=dev)
+    rid = torch.randperm(16384, generator=g_sr, device=dev)[:8192].contiguous()
+    qkr.rope_set_rows(k, cache, rid, pos4, inv4, 128, W.SECTIONS_INTERLEAVED, (24, 20, 20), 0,
+                      stream=stream)
+    torch.cuda.synchronize()
+    kw4 = W.RopeWorkload("k", [W.StreamInputs(s4.k, s4.k, s4.gamma_k, s4.gamma_k)], 8, 8,
+                         w4.D, w4.rot, w4.pairing, w4.eps, w4.angle, norm=False)
+    got = cache[rid[:S]].cpu()
+    legs["K 8192 x 8 heads x 128 -> 16384-row cache, interleaved (24,20,20)"] = _leg_rope(
+        kw4, got, got, list(range(S)),
+        lambda a, b: [W.StreamInputs(s4.k[a:b], s4.k[a:b], s4.gamma_k, s4.gamma_k)],
+        pos_at, "cache rows of tokens 0..%d" % (S - 1))
+    del cache, q, k
+
+    # config 5: ViT setup (all planes) and apply
+    w5 = W.config5()
+    gr = np.asarray(w5.grids, dtype=np.int64)
+    cu = np.concatenate([[0], np.cumsum(gr[:, 0] * gr[:, 1] * gr[:, 2])])
+    N = int(cu[-1])
+    meta = torch.from_numpy(np.concatenate([cu, gr.reshape(-1)]).astype(np.int32)).to(dev)
+    G = len(w5.grids)
+    cos5 = torch.full((3, N, 64), float("nan"), dtype=torch.float32, device=dev)
+    sin5 = torch.full_like(cos5, float("nan"))
+    qkr.vit_mrope_setup(w5.inv_t.to(dev), w5.inv_h.to(dev), w5.inv_w.to(dev), meta[:G + 1],
+                        meta[G + 1:].view(G, 3), N, 2, cos5, sin5, stream)
+    torch.cuda.synchronize()
+    pos = oracle.vit_positions(w5.grids, 2)
+    rc, rs, written = oracle.vit_planes(pos, w5.inv_t, w5.inv_h, w5.inv_w)
+    mask = written.astype(bool)
+    gc, gs = cos5.cpu().numpy(), sin5.cpu().numpy()
+    gv = np.concatenate([gc[mask], gs[mask]]).astype(np.float64)
+    rv = np.concatenate([rc[mask], rs[mask]]).astype(np.float64)
+    rel = np.abs(gv - rv) / np.maximum(np.abs(rv), 1e-30)
+    err = {"elements": int(rv.size), "max_rel": float(rel.max()),
+           "outside_tolerance": int((~(np.abs(gv - rv) <= 2e-6 * np.abs(rv))).sum()),
+           "unwritten_cells_untouched": bool(np.isnan(gc[~mask]).all() and
+                                             np.isnan(gs[~mask]).all()),
+           "sample": "every written cell of the (3, N, 64) planes"}
+    single, allc = _time_leg(
+        lambda: oracle.vit_planes(oracle.vit_positions(w5.grids, 2), w5.inv_t, w5.inv_h,
+                                  w5.inv_w), N,
+        [(lambda g_=g_: oracle.vit_planes(oracle.vit_positions([g_], 2), w5.inv_t, w5.inv_h,
+                                          w5.inv_w), int(g_[0] * g_[1] * g_[2]))
+         for g_ in w5.grids], "tokens", "all %d tokens (positions + planes)" % N)
+    legs["8 grids N=%d, planes (3,N,64) fp32" % N] = {
+        "cpu_baseline": single, "cpu_baseline_all_cores": allc, "error_vs_oracle": err}
+    q5, k5 = w5.q.to(dev), w5.k.to(dev)
+    qo5, ko5 = torch.empty_like(q5), torch.empty_like(k5)
+    a5 = qkr.angle_table(cos5, sin5, W.SECTIONS_CONTIGUOUS, (16, 24, 24))
+    qkr.fused_qk_norm_rope([(q5, k5, w5.gamma_q.to(dev), w5.gamma_k.to(dev))], qo5, ko5, 64, 0,
+                           1e-6, a5, 0, stream)
+    torch.cuda.synchronize()
+    A5 = W.AngleInputs(kind=W.ANGLE_TABLE, section_mode=W.SECTIONS_CONTIGUOUS,
+                       sections=(16, 24, 24, 0), cos=rc, sin=rs)
+    w5r = W.RopeWorkload("vit", [W.StreamInputs(w5.q, w5.k, w5.gamma_q, w5.gamma_k)], 16, 16,
+                         80, 64, W.PAIRING_NEOX, 1e-6, A5)
+
+    def planes_at(a):
+        return W.AngleInputs(kind=W.ANGLE_TABLE, section_mode=W.SECTIONS_CONTIGUOUS,
+                             sections=(16, 24, 24, 0), cos=rc, sin=rs, token_offset=a)
+    legs["ViT apply N=%d H=16 D=80 rot=64 from the 3 planes" % N] = _leg_rope(
+        w5r, qo5.cpu(), ko5.cpu(), list(range(S)),
+        lambda a, b: [W.StreamInputs(w5.q[a:b], w5.k[a:b], w5.gamma_q, w5.gamma_k)],
+        planes_at, "tokens 0..%d" % (S - 1))
+    del q5, k5, cos5, sin5
+
+    # config 2: RMSNorm + residual (and the FP8 output) on sampled rows
+    for R, hidden in [(1, 5120), (32, 5120), (1024, 8192), (4096, 8192), (16384, 8192),
+                      (16384, 2048)]:
+        w2 = W.config2(R=R, hidden=hidden)
+        n = min(R, LEG_ROWS)
+        x, r0, gm = w2.x.to(dev), w2.residual.to(dev), w2.gamma.to(dev)
+        res, out = r0.clone(), torch.empty_like(x)
+        qkr.rms_norm_residual(x, res, gm, out, 1e-6, stream)
+        torch.cuda.synchronize()
+        xs, rs_, gs_ = w2.x[:n], w2.residual[:n], w2.gamma
+
+        def run_rows(a, b, xs=xs, rs_=rs_, gs_=gs_):
+            return oracle.rms_norm_residual(xs[a:b], rs_[a:b], gs_, 1e-6)
+        ro, oo = run_rows(0, n)
+        err = _err_report(out[:n].float().cpu().numpy().astype(np.float64), oo,
+                          "rows 0..%d" % (n - 1))
+        err["residual_bit_exact"] = bool(np.array_equal(oracle.bits(res[:n].cpu()), ro))
+        single, allc = _time_leg(lambda: run_rows(0, n), n,
+                                 _token_slices(lambda a, b: (lambda: run_rows(a, b)), n, 64),
+                                 "rows", "rows 0..%d" % (n - 1))
+        legs["R=%d hidden=%d" % (R, hidden)] = {"cpu_baseline": single,
+                                                 "cpu_baseline_all_cores": allc,
+                                                 "error_vs_oracle": err}
+        if R in (1, 1024, 16384) and hidden == 8192 or R == 1:
+            sc = torch.tensor([0.05], dtype=torch.float32, device=dev)
+            res8, o8 = r0.clone(), torch.empty(R, hidden, dtype=torch.uint8, device=dev)
+            qkr.rms_norm_fp8(x, res8, gm, o8, sc, 1e-6, stream)
+            torch.cuda.synchronize()
+
+            def run8(a, b, xs=xs, rs_=rs_, gs_=gs_):
+                return oracle.rms_norm_fp8(xs[a:b], rs_[a:b], gs_, 1e-6, 0.05)
+            r8, y8, c8 = run8(0, n)
+            codes = o8[:n].cpu().numpy()
+            single, allc = _time_leg(lambda: run8(0, n), n,
+                                     _token_slices(lambda a, b: (lambda: run8(a, b)), n, 64),
+                                     "rows", "rows 0..%d" % (n - 1))
+            legs["R=%d hidden=%d, FP8 E4M3 out" % (R, hidden)] = {
+                "cpu_baseline": single, "cpu_baseline_all_cores": allc,
+                "error_vs_oracle": {"elements": int(codes.size),
+                                    "codes_equal": int((codes == c8).sum()),
+                                    "residual_bit_exact": bool(np.array_equal(
+                                        oracle.bits(res8[:n].cpu()), r8)),
+                                    "sample": "rows 0..%d" % (n - 1)}}
+        del x, r0, res, out
+    torch.cuda.empty_cache()
+    return legs
 
 
 def reference_arm(args) -> dict:
@@ -738,9 +1059,13 @@ def main():
         sweep = rms_sweep(dev, stream, peaks["hbm_gbs"])
 
     cb = cbp = None
+    legs = {}
     if rank == 0 and world == 1 and not args.no_cpu:
         cb = cpu_baseline()
         cbp = cpu_baseline_parallel()
+        legs = oracle_legs(dev, stream)
+        for r in rows:
+            r.update(legs.get(r["workload"], {}))
 
     if dist:
         dist.barrier()
@@ -781,6 +1106,7 @@ def main():
                      "kernel": info.get("kernel_name")},
         "cpu_baseline": cb,
         "cpu_baseline_all_cores": cbp,
+        "error_vs_oracle": legs.get("headline", {}).get("error_vs_oracle"),
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "path": "pinned host -> H2D stream | fused_qk_norm_rope stream | D2H stream "

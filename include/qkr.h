@@ -14,7 +14,7 @@
  *   vit_mrope_setup     fp32 (3, N, P) cos/sin t/h/w planes computed from
  *                       per-image [t, h, w] grids.
  *   rms_norm_residual   hidden-size RMSNorm with a fused residual add; splits
- *                       one row across a thread-block cluster when rows are few.
+ *                       a wide row across a thread-block cluster when rows are few.
  *   rms_norm_fp8        the same with a static-scale FP8 E4M3 output.
  *   rope_set_rows       mrope_apply's rotation of K rows, scattered into cache
  *                       rows by index.
@@ -100,13 +100,38 @@ enum {
     QKR_ANGLE_TABLE = 1
 };
 
-/* Flags for fused_qk_norm_rope / mrope_apply. */
+/* Flags for fused_qk_norm_rope / fused_qkv_norm_rope / mrope_apply /
+ * rope_set_rows.  The first two set the rounding points of the normalised
+ * value: without either, every intermediate stays in fp32 (gamma folded into
+ * the rotation) and only the output is rounded; at most one of them, and
+ * either needs the norm. */
 enum {
     /* Round the normalised value to bf16 before rotating (the rounding
      * contract of the vllm-omni #7600 Triton tile: bf16-rounded normalised
-     * value, fp32 rotation, one final rounding).  Without the flag every
-     * intermediate stays in fp32 and only the output is rounded. */
-    QKR_FLAG_ROUND_NORMALIZED_BF16 = 1u
+     * value, fp32 rotation, one final rounding). */
+    QKR_FLAG_ROUND_NORMALIZED_BF16 = 1u,
+    /* The eager chain's rounding points (vllm-omni #7600, numerics follow-up:
+     * a preset that reproduces the unfused RMSNorm and RoPE chain; vLLM
+     * #26234 quotes the rms_norm_kernel line that fixes them): the normalised
+     * value x r (r = rsqrt(mean(x^2) + eps), fp32) is rounded to bf16, its
+     * product with the bf16 gamma is rounded to bf16 again, and the rotation
+     * a c - b s, b c + a s takes every product and sum in fp32 without fused
+     * multiply-adds; one final rounding.  The rounding points, not bitwise
+     * equality with any other implementation: the order of the fp32 sum of
+     * squares is this library's. */
+    QKR_FLAG_EAGER_ROUNDING = 2u,
+    /* A launch-order contract, not a rounding point: the caller declares
+     * that this call reads no memory the previous kernel on the stream
+     * writes, and writes no memory that kernel reads or writes (the chunks
+     * of one chunked step, llama.cpp fork #286, "The change": a launch over
+     * part of the tokens).  The kernel then starts its rows while the
+     * previous kernel's last CTAs drain (with qkr_launch_overlap on) and
+     * waits for that kernel only before it completes, so everything after
+     * it on the stream still sees the writes of both.  Results are
+     * bit-identical with and without the flag; a call that breaks the
+     * contract races with the previous kernel.  Combines with either
+     * rounding flag. */
+    QKR_FLAG_INDEPENDENT = 4u
 };
 
 /* One input stream of fused_qk_norm_rope / fused_qkv_norm_rope.  q, k and v
@@ -180,7 +205,8 @@ typedef struct qkr_angle_desc {
  *                    Fresh outputs: they must not overlap any input.
  *   D                head dim, a multiple of 8, 8 <= D <= 256.
  *   rot_dim          even, 0 <= rot_dim <= D.
- *   flags            0 or QKR_FLAG_ROUND_NORMALIZED_BF16.
+ *   flags            0, QKR_FLAG_ROUND_NORMALIZED_BF16 or QKR_FLAG_EAGER_ROUNDING,
+ *                    optionally with QKR_FLAG_INDEPENDENT.
  * Alignment: q/k (after offsets), gammas and outputs 16-byte aligned; all
  * token and head strides multiples of 8 elements (else QKR_ERR_UNSUPPORTED).
  */
@@ -305,10 +331,11 @@ qkr_status vit_mrope_setup(void *stream, const float *inv_t, const float *inv_h,
  * (vllm.cpp #185, "decode RmsNorm ran on ONE workgroup"; vLLM #26234
  * rms_norm_kernel): per row, s = bf16(x + residual) is written back to
  * residual, then out = s / sqrt(mean(s^2) + eps) * gamma (fp32 sum of
- * squares, one final bf16 rounding).  When rows are too few to fill the GPU
- * (decode: up to 32 rows) each row is split across a thread-block cluster of
- * 8 (up to 8 rows) or 4 CTAs whose partial sums meet in distributed shared
- * memory.
+ * squares, one final bf16 rounding).  A row that fits one CTA (hidden <=
+ * 8192) is one CTA wide enough to have every 16-byte vector of the row in
+ * flight at once; a wider row at decode sizes (up to 32 rows) is split
+ * across a thread-block cluster of 8 (up to 16 rows) or 4 CTAs whose partial
+ * sums meet in distributed shared memory.
  *
  *   x                bf16 device [R, hidden], row stride x_stride.
  *   residual         bf16 device [R, hidden], in/out, row stride res_stride.

@@ -23,6 +23,8 @@ PAIRING_NEOX, PAIRING_GPTJ = 0, 1
  SECTIONS_IMROPE) = range(5)
 ANGLE_POSITIONS, ANGLE_TABLE = 0, 1
 FLAG_ROUND_NORMALIZED_BF16 = 1
+FLAG_EAGER_ROUNDING = 2
+FLAG_INDEPENDENT = 4
 KERNEL_NAMES = {0: "none", 1: "rope_paired", 2: "rope_vector", 3: "rope_exchange",
                 4: "vit_setup", 5: "rms_rows", 6: "rms_cluster", 7: "section_map",
                 8: "vit_positions", 9: "null"}

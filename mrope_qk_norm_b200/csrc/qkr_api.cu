@@ -242,8 +242,14 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
         return fail(QKR_ERR_INVALID_ARG, "V head count out of range");
     if (!streams || n_streams < 1 || n_streams > 2)
         return fail(QKR_ERR_INVALID_ARG, "need 1 or 2 stream descriptors");
-    if (flags & ~(uint32_t)QKR_FLAG_ROUND_NORMALIZED_BF16)
+    if (flags & ~(uint32_t)(QKR_FLAG_ROUND_NORMALIZED_BF16 | QKR_FLAG_EAGER_ROUNDING |
+                            QKR_FLAG_INDEPENDENT))
         return fail(QKR_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & QKR_FLAG_ROUND_NORMALIZED_BF16) && (flags & QKR_FLAG_EAGER_ROUNDING))
+        return fail(QKR_ERR_INVALID_ARG, "one rounding contract at a time: ROUND_NORMALIZED_BF16 "
+                                         "or EAGER_ROUNDING");
+    if (!norm && (flags & (QKR_FLAG_ROUND_NORMALIZED_BF16 | QKR_FLAG_EAGER_ROUNDING)))
+        return fail(QKR_ERR_INVALID_ARG, "the rounding contracts need normalisation (gammas)");
     int64_t T_all = 0;
     for (int s = 0; s < n_streams; ++s) {
         if (streams[s].n_tokens < 0 || streams[s].n_tokens > ((int64_t)1 << 40))
@@ -433,7 +439,10 @@ qkr_status rope_call(void *stream, const qkr_stream_desc *streams, int32_t n_str
     p.eps = eps;
     p.inv_D = 1.0f / (float)D;
     p.norm = norm ? 1 : 0;
-    p.round_norm = (flags & QKR_FLAG_ROUND_NORMALIZED_BF16) ? 1 : 0;
+    p.independent = (flags & QKR_FLAG_INDEPENDENT) ? 1 : 0;
+    p.round_norm = (flags & QKR_FLAG_EAGER_ROUNDING)          ? 2   // kRoundEager
+                 : (flags & QKR_FLAG_ROUND_NORMALIZED_BF16) ? 1   // kRoundNormalized
+                                                            : 0;
 
     qkr::LaunchRecord rec;
     cudaError_t e = qkr::launch_rope_rows(p, pairing, static_cast<cudaStream_t>(stream), &rec);
@@ -575,8 +584,8 @@ qkr_status mrope_apply(void *stream, const void *q, const void *k, void *q_out, 
     if ((gamma_q == nullptr) != (gamma_k == nullptr))
         return fail(QKR_ERR_INVALID_ARG, "gamma_q and gamma_k must be both set or both NULL");
     const bool norm = gamma_q != nullptr;
-    if (!norm && (flags & QKR_FLAG_ROUND_NORMALIZED_BF16))
-        return fail(QKR_ERR_INVALID_ARG, "ROUND_NORMALIZED_BF16 needs normalisation (gammas)");
+    if (!norm && (flags & (QKR_FLAG_ROUND_NORMALIZED_BF16 | QKR_FLAG_EAGER_ROUNDING)))
+        return fail(QKR_ERR_INVALID_ARG, "the rounding contracts need normalisation (gammas)");
     if (section_mode < QKR_SECTIONS_NONE || section_mode > QKR_SECTIONS_IMROPE)
         return fail(QKR_ERR_INVALID_ARG, "unknown section mode %d", section_mode);
     if (rot_dim > 0 && n_rows != rows_for_mode(section_mode))
@@ -641,8 +650,8 @@ qkr_status rope_set_rows(void *stream, const void *x, void *cache, const int64_t
                          int32_t pairing, const void *gamma, float eps, uint32_t flags)
 {
     const bool norm = gamma != nullptr;
-    if (!norm && (flags & QKR_FLAG_ROUND_NORMALIZED_BF16))
-        return fail(QKR_ERR_INVALID_ARG, "ROUND_NORMALIZED_BF16 needs normalisation (gamma)");
+    if (!norm && (flags & (QKR_FLAG_ROUND_NORMALIZED_BF16 | QKR_FLAG_EAGER_ROUNDING)))
+        return fail(QKR_ERR_INVALID_ARG, "the rounding contracts need normalisation (gamma)");
     if (section_mode < QKR_SECTIONS_NONE || section_mode > QKR_SECTIONS_IMROPE)
         return fail(QKR_ERR_INVALID_ARG, "unknown section mode %d", section_mode);
     if (rot_dim > 0 && n_rows != rows_for_mode(section_mode))

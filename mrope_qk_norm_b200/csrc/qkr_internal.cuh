@@ -78,6 +78,28 @@ __device__ __forceinline__ void pdl_trigger()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The rope kernels' entry and exit under QKR_FLAG_INDEPENDENT.  A call the
+// caller declares independent of the previous kernel on the stream (it reads
+// nothing that kernel writes, writes nothing it reads or writes) starts its
+// work without the grid-dependency wait, so its CTAs stream their rows while
+// the previous kernel's last CTAs drain, and takes the wait just before it
+// exits instead: it cannot complete before the previous kernel has, so every
+// kernel after it still sees the writes of both.  The previous kernel's CTAs
+// have all started when this one launches (each triggers its dependents
+// first thing), so a CTA waiting at the end never holds an SM that the
+// previous kernel still needs.
+__device__ __forceinline__ void pdl_enter(int independent)
+{
+    if (!independent)
+        pdl_wait();
+    pdl_trigger();
+}
+__device__ __forceinline__ void pdl_exit(int independent)
+{
+    if (independent)
+        pdl_wait();
+}
+
 // Process-wide switch (qkr_launch_overlap); 1 = launch with the attribute.
 int launch_overlap();
 void set_launch_overlap(int enable);
@@ -179,6 +201,7 @@ struct RopeParams {
     int64_t k_out_rows;       // scatter: rows of k_out
     unsigned *status;         // device status word (scatter: out-of-range rows)
     int stages;               // streaming kernel: depth of the cp.async row ring
+    int independent;          // QKR_FLAG_INDEPENDENT: wait for the previous grid at the end
     int64_t token_offset;
 };
 

@@ -228,20 +228,32 @@ cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, La
 {
     const bool fp8 = p.out8 != nullptr;
     const int nvec = p.hidden >> 3;
-    // CTAs per row.  A sweep on B200 (hidden 5120 / 8192, R = 1 .. 128) put the
-    // best split at 8 CTAs for up to 8 rows, 4 for up to 32 and one CTA per row
-    // beyond: a cluster launch and its DSMEM exchange cost more than the extra
-    // SMs save once a few rows are in flight (R = 32: 2.61 us at 4 per row vs
-    // 3.54 us at 16; R = 128: 3.98 us at 1 vs 4.81 us at 4).  A slice keeps at
-    // least 32 vectors per CTA.
-    int cs = p.R <= 8 ? 8 : (p.R <= 32 ? 4 : 1);
+    // CTAs per row and threads per CTA, from sweeps on B200 (R = 1 .. 4096,
+    // hidden 2048 .. 65536, graph-replayed back-to-back launches):
+    //   * one CTA per row whenever a row fits one CTA (hidden <= 8192): every
+    //     vector of the row in flight at once beats a cluster split, whose
+    //     launch and DSMEM exchange cost ~0.9 us (R = 1 x 2048: 1.28 us
+    //     against 2.13 us split over 8 CTAs; R = 1 x 5120: 1.66 against 2.21);
+    //   * wider rows at decode sizes split over a cluster: 8 CTAs up to 16
+    //     rows, 4 up to 32 (R = 1 x 65536: 3.3 us against 11.3 us in one CTA);
+    //   * width: one vector per thread for up to 128 rows (up to 1024
+    //     threads), two per thread beyond (R = 1024 x 8192: 12.0 us at 512
+    //     threads against 12.4 at 256 and 13.7 at 1024).
+    // A cluster slice keeps at least 32 vectors per CTA.
+    int cs = 1;
+    if (nvec > 1024 && p.R <= 32)
+        cs = p.R <= 16 ? 8 : 4;
     while (cs > 1 && nvec / cs < 32)
         cs >>= 1;
     if (g_force_cluster > 0 && nvec / g_force_cluster >= 1)
         cs = g_force_cluster;
     int vpt, threads;
     const int per = (nvec + cs - 1) / cs;
-    const int target = g_force_threads > 0 ? (int)g_force_threads : 256;
+    int target = cs == 8 ? 512 : (p.R <= 128 ? 1024 : (per + 1) / 2);
+    if (target < 32)
+        target = 32;
+    if (g_force_threads > 0)
+        target = g_force_threads;
     shape(per, target, vpt, threads);
     if ((int64_t)threads * vpt < per)
         return cudaErrorInvalidConfiguration;

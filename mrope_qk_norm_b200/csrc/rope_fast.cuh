@@ -49,10 +49,10 @@ using KernelFn = void (*)(RopeParams);
 // Pickers exported by the instantiation units: layout and angle path (staged
 // or direct) fixed by the unit; lanes per row, slots, heads per item and the
 // norm flags chosen at run time.
-KernelFn pick_fast_paired_staged(int lpr, int ns, int u, bool norm, bool round);
-KernelFn pick_fast_paired_direct(int lpr, int ns, int u, bool norm, bool round);
-KernelFn pick_fast_vector_staged(int lpr, int ns, int u, bool norm, bool round);
-KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, bool round);
+KernelFn pick_fast_paired_staged(int lpr, int ns, int u, bool norm, int rmode);
+KernelFn pick_fast_paired_direct(int lpr, int ns, int u, bool norm, int rmode);
+KernelFn pick_fast_vector_staged(int lpr, int ns, int u, bool norm, int rmode);
+KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, int rmode);
 
 namespace {
 
@@ -214,12 +214,11 @@ __device__ __forceinline__ void copy_v_rows(const RopeParams &p, int64_t tok0, i
     }
 }
 
-template <int LAYOUT, int LPR, int NS, int U, bool NORM, bool ROUND, bool DIRECT>
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE, bool DIRECT>
 __global__ void __launch_bounds__(kThreads)
 rope_fast_kernel(const __grid_constant__ RopeParams p)
 {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter(p.independent);
     // Quads (couples of pairs) per lane: PAIRED lo/hi vectors hold 4, each
     // VECTOR slot holds 2.  Pass-through slots (PAIRED tail) are scaled only.
     constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
@@ -321,7 +320,7 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
                 gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
             unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
         }
-        RotCoef<NQ, NORM && !ROUND> kc;
+        RotCoef<NQ, NORM && RMODE == kRoundNone> kc;
         make_coef(kc, C, Sn, GA, GB);
 
 #pragma unroll
@@ -336,7 +335,7 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
                     ss += __shfl_xor_sync(0xffffffffu, ss, off);
                 r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
             }
-            norm_rotate<LAYOUT, NS, NORM, ROUND>(A, B, TL, r, kc, GA, GB, GT);
+            norm_rotate<LAYOUT, NS, NORM, RMODE>(A, B, TL, r, kc, GA, GB, GT);
             uint4 outv[NS];
             pack_row<LAYOUT, NS>(A, B, TL, outv);
             if (u < m.nh) {
@@ -347,60 +346,66 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
             }
         }
     }
+    pdl_exit(p.independent);
 }
 
 // ------------------------------------------------------------- pickers --
 
 template <int LAYOUT, bool DIRECT, int LPR, int NS, int U>
-KernelFn pick_flags(bool norm, bool round)
+KernelFn pick_flags(bool norm, int rmode)
 {
     if (!norm)
-        return rope_fast_kernel<LAYOUT, LPR, NS, U, false, false, DIRECT>;
-    return round ? rope_fast_kernel<LAYOUT, LPR, NS, U, true, true, DIRECT>
-                 : rope_fast_kernel<LAYOUT, LPR, NS, U, true, false, DIRECT>;
+        return rope_fast_kernel<LAYOUT, LPR, NS, U, false, kRoundNone, DIRECT>;
+    switch (rmode) {
+    case kRoundNone: return rope_fast_kernel<LAYOUT, LPR, NS, U, true, kRoundNone, DIRECT>;
+    case kRoundNormalized:
+        return rope_fast_kernel<LAYOUT, LPR, NS, U, true, kRoundNormalized, DIRECT>;
+    case kRoundEager: return rope_fast_kernel<LAYOUT, LPR, NS, U, true, kRoundEager, DIRECT>;
+    default: return nullptr;
+    }
 }
 
 template <int LAYOUT, bool DIRECT, int LPR, int NS>
-KernelFn pick_u(int u, bool norm, bool round)
+KernelFn pick_u(int u, bool norm, int rmode)
 {
     switch (u) {
-    case 1: return pick_flags<LAYOUT, DIRECT, LPR, NS, 1>(norm, round);
-    case 2: return pick_flags<LAYOUT, DIRECT, LPR, NS, 2>(norm, round);
-    case 3: return pick_flags<LAYOUT, DIRECT, LPR, NS, 3>(norm, round);
-    case 4: return pick_flags<LAYOUT, DIRECT, LPR, NS, 4>(norm, round);
+    case 1: return pick_flags<LAYOUT, DIRECT, LPR, NS, 1>(norm, rmode);
+    case 2: return pick_flags<LAYOUT, DIRECT, LPR, NS, 2>(norm, rmode);
+    case 3: return pick_flags<LAYOUT, DIRECT, LPR, NS, 3>(norm, rmode);
+    case 4: return pick_flags<LAYOUT, DIRECT, LPR, NS, 4>(norm, rmode);
     default: return nullptr;
     }
 }
 
 template <int LAYOUT, bool DIRECT, int LPR>
-KernelFn pick_ns(int ns, int u, bool norm, bool round)
+KernelFn pick_ns(int ns, int u, bool norm, int rmode)
 {
     if constexpr (LAYOUT == PAIRED) {
         // slots 0/1: the two rotary halves of the lane's pairs; 2, 3: pass-through tail
         switch (ns) {
-        case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, round);
-        case 3: return pick_u<LAYOUT, DIRECT, LPR, 3>(u, norm, round);
-        case 4: return pick_u<LAYOUT, DIRECT, LPR, 4>(u, norm, round);
+        case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, rmode);
+        case 3: return pick_u<LAYOUT, DIRECT, LPR, 3>(u, norm, rmode);
+        case 4: return pick_u<LAYOUT, DIRECT, LPR, 4>(u, norm, rmode);
         default: return nullptr;
         }
     } else {
         switch (ns) {
-        case 1: return pick_u<LAYOUT, DIRECT, LPR, 1>(u, norm, round);
-        case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, round);
+        case 1: return pick_u<LAYOUT, DIRECT, LPR, 1>(u, norm, rmode);
+        case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, rmode);
         default: return nullptr;
         }
     }
 }
 
 template <int LAYOUT, bool DIRECT>
-KernelFn pick_fast(int lpr, int ns, int u, bool norm, bool round)
+KernelFn pick_fast(int lpr, int ns, int u, bool norm, int rmode)
 {
     switch (lpr) {
-    case 1: return pick_ns<LAYOUT, DIRECT, 1>(ns, u, norm, round);
-    case 2: return pick_ns<LAYOUT, DIRECT, 2>(ns, u, norm, round);
-    case 4: return pick_ns<LAYOUT, DIRECT, 4>(ns, u, norm, round);
-    case 8: return pick_ns<LAYOUT, DIRECT, 8>(ns, u, norm, round);
-    case 16: return pick_ns<LAYOUT, DIRECT, 16>(ns, u, norm, round);
+    case 1: return pick_ns<LAYOUT, DIRECT, 1>(ns, u, norm, rmode);
+    case 2: return pick_ns<LAYOUT, DIRECT, 2>(ns, u, norm, rmode);
+    case 4: return pick_ns<LAYOUT, DIRECT, 4>(ns, u, norm, rmode);
+    case 8: return pick_ns<LAYOUT, DIRECT, 8>(ns, u, norm, rmode);
+    case 16: return pick_ns<LAYOUT, DIRECT, 16>(ns, u, norm, rmode);
     default: return nullptr;
     }
 }

@@ -4,9 +4,9 @@
 
 namespace qkr {
 
-KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, bool round)
+KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, int rmode)
 {
-    return pick_fast<VECTOR, true>(lpr, ns, u, norm, round);
+    return pick_fast<VECTOR, true>(lpr, ns, u, norm, rmode);
 }
 
 }  // namespace qkr

@@ -113,7 +113,7 @@ __device__ __forceinline__ float row_sumsq(const float2 (&A)[RowShape<LAYOUT, NS
 }
 
 // Per-work-item coefficients of the rotation (see the header comment).
-// FOLD (norm without the bf16-rounded-normalised contract): K0 = g_a c,
+// FOLD (norm with no intermediate rounding, kRoundNone): K0 = g_a c,
 // K1 = -(g_b s), K2 = g_b c, K3 = g_a s.  Otherwise K0 = c, K1 = -s, K2 = c,
 // K3 = s, and GA / GB keep the gammas for the explicit normalisation.
 template <int NQ, bool FOLD>
@@ -143,13 +143,25 @@ __device__ __forceinline__ void make_coef(RotCoef<NQ, FOLD> &k, const float2 (&C
     }
 }
 
+// Rounding points of the normalised value (RMODE; RopeParams::round_norm):
+//   kRoundNone       y = x r gamma stays fp32 (gamma folded into the rotation
+//                    coefficients), the rotation is fused multiply-adds, and
+//                    only the output is rounded;
+//   kRoundNormalized y = bf16(x r gamma) before an fp32 rotation
+//                    (QKR_FLAG_ROUND_NORMALIZED_BF16);
+//   kRoundEager      y = bf16(bf16(x r) gamma) -- the eager RMSNorm casts the
+//                    normalised value to bf16, then multiplies by the bf16
+//                    weight -- and the rotation's products and sums are each
+//                    rounded to fp32, with no contraction into fused
+//                    multiply-adds (QKR_FLAG_EAGER_ROUNDING).
+enum { kRoundNone = 0, kRoundNormalized = 1, kRoundEager = 2 };
+
 // Normalise (NORM: by r and gamma) and rotate one row's couples in place.
-// ROUND: the normalised value is rounded to bf16 before the rotation.
-template <int LAYOUT, int NS, bool NORM, bool ROUND>
+template <int LAYOUT, int NS, bool NORM, int RMODE>
 __device__ __forceinline__ void norm_rotate(
     float2 (&A)[RowShape<LAYOUT, NS>::NQ], float2 (&B)[RowShape<LAYOUT, NS>::NQ],
     float2 (&T)[RowShape<LAYOUT, NS>::NTA][4], float r,
-    const RotCoef<RowShape<LAYOUT, NS>::NQ, NORM && !ROUND> &k,
+    const RotCoef<RowShape<LAYOUT, NS>::NQ, NORM && RMODE == kRoundNone> &k,
     const float2 (&GA)[RowShape<LAYOUT, NS>::NQ], const float2 (&GB)[RowShape<LAYOUT, NS>::NQ],
     const float2 (&GT)[RowShape<LAYOUT, NS>::NTA][4])
 {
@@ -159,13 +171,24 @@ __device__ __forceinline__ void norm_rotate(
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
         float2 a = A[q], b = B[q];
-        if (NORM && ROUND) {
+        if (NORM && RMODE == kRoundNormalized) {
             a = round2_bf16(__fmul2_rn(__fmul2_rn(a, r2), GA[q]));
             b = round2_bf16(__fmul2_rn(__fmul2_rn(b, r2), GB[q]));
         }
-        float2 a2 = __ffma2_rn(b, k.K1[q], __fmul2_rn(a, k.K0[q]));
-        float2 b2 = __ffma2_rn(a, k.K3[q], __fmul2_rn(b, k.K2[q]));
-        if (NORM && !ROUND) {
+        if (NORM && RMODE == kRoundEager) {
+            a = round2_bf16(__fmul2_rn(round2_bf16(__fmul2_rn(a, r2)), GA[q]));
+            b = round2_bf16(__fmul2_rn(round2_bf16(__fmul2_rn(b, r2)), GB[q]));
+        }
+        float2 a2, b2;
+        if (RMODE == kRoundEager) {
+            // K1 = -s: a c + b (-s) is a c - b s with every step rounded
+            a2 = __fadd2_rn(__fmul2_rn(a, k.K0[q]), __fmul2_rn(b, k.K1[q]));
+            b2 = __fadd2_rn(__fmul2_rn(b, k.K2[q]), __fmul2_rn(a, k.K3[q]));
+        } else {
+            a2 = __ffma2_rn(b, k.K1[q], __fmul2_rn(a, k.K0[q]));
+            b2 = __ffma2_rn(a, k.K3[q], __fmul2_rn(b, k.K2[q]));
+        }
+        if (NORM && RMODE == kRoundNone) {
             a2 = __fmul2_rn(a2, r2);
             b2 = __fmul2_rn(b2, r2);
         }
@@ -177,7 +200,10 @@ __device__ __forceinline__ void norm_rotate(
         for (int t = 0; t < NT; ++t)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                T[t][i] = __fmul2_rn(__fmul2_rn(T[t][i], r2), GT[t][i]);
+                T[t][i] = RMODE == kRoundEager
+                              ? round2_bf16(__fmul2_rn(round2_bf16(__fmul2_rn(T[t][i], r2)),
+                                                       GT[t][i]))
+                              : __fmul2_rn(__fmul2_rn(T[t][i], r2), GT[t][i]);
     }
 }
 

@@ -24,8 +24,7 @@ template <int LPR, int NS>
 __global__ void __launch_bounds__(kThreads)
 rope_exchange_kernel(const __grid_constant__ RopeParams p)
 {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter(p.independent);
     constexpr int G = kThreads / LPR;
     extern __shared__ float4 smem[];
     const int cs_ld = (p.pw + 3) & ~3;
@@ -109,8 +108,12 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
                 unpack8(ld_reuse(gam + 8 * vidx[k]), g);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    x[k][e] = (x[k][e] * inv_rms) * g[e];
-                    if (p.round_norm)
+                    if (p.round_norm == kRoundEager)
+                        x[k][e] = round_bf16(__fmul_rn(round_bf16(__fmul_rn(x[k][e], inv_rms)),
+                                                       g[e]));
+                    else
+                        x[k][e] = (x[k][e] * inv_rms) * g[e];
+                    if (p.round_norm == kRoundNormalized)
                         x[k][e] = round_bf16(x[k][e]);
                 }
             }
@@ -135,8 +138,12 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
                     const bool lo = el < half;
                     const int j = lo ? el : el - half;
                     const float other = xbuf[lo ? el + half : el - half];
-                    x[k][e] = lo ? x[k][e] * cr[j] - other * sr[j]
-                                 : x[k][e] * cr[j] + other * sr[j];
+                    if (p.round_norm == kRoundEager)  // every product and sum rounded
+                        x[k][e] = lo ? __fsub_rn(__fmul_rn(x[k][e], cr[j]), __fmul_rn(other, sr[j]))
+                                     : __fadd_rn(__fmul_rn(x[k][e], cr[j]), __fmul_rn(other, sr[j]));
+                    else
+                        x[k][e] = lo ? x[k][e] * cr[j] - other * sr[j]
+                                     : x[k][e] * cr[j] + other * sr[j];
                 }
             }
         }
@@ -148,6 +155,7 @@ rope_exchange_kernel(const __grid_constant__ RopeParams p)
                     st_stream(dst + 8 * vidx[k], isv ? raw[k] : pack8(x[k]));
         }
     }
+    pdl_exit(p.independent);
 }
 
 // ================================================================== host ==
@@ -280,7 +288,10 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
     // 8192 and 5735 tokens were fastest at 8 and one of 2457 at 4 (8.5 us
     // against 9.3 us at 8, whose grid is half a wave); 16 tokens per CTA
     // was 8-13% slower on all three (each CTA's staging prologue is exposed
-    // once per range, over fewer CTAs).
+    // once per range, over fewer CTAs).  Whole waves of balanced ranges
+    // (grid a multiple of the resident CTAs, at most 8 tokens each) were
+    // slower still: the chunked pair took 24.35 us against 23.96 us, more
+    // CTAs paying the prologue costing more than the partly filled last wave.
     int64_t grid;
     int tt = g_force_tt;
     if (tt <= 0) {
@@ -438,14 +449,15 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     int best_u = layout == EXCHANGE ? 1 : direct ? (ns <= 3 ? 4 : 2) : 2;
     if (g_force_u > 0 && layout != EXCHANGE)
         best_u = g_force_u;
-    const bool norm = p.norm != 0, round = p.round_norm != 0;
+    const bool norm = p.norm != 0;
+    const int rmode = p.round_norm;
     KernelFn fn;
     if (layout == PAIRED)
-        fn = direct ? pick_fast_paired_direct(lpr, ns, best_u, norm, round)
-                    : pick_fast_paired_staged(lpr, ns, best_u, norm, round);
+        fn = direct ? pick_fast_paired_direct(lpr, ns, best_u, norm, rmode)
+                    : pick_fast_paired_staged(lpr, ns, best_u, norm, rmode);
     else if (layout == VECTOR)
-        fn = direct ? pick_fast_vector_direct(lpr, ns, best_u, norm, round)
-                    : pick_fast_vector_staged(lpr, ns, best_u, norm, round);
+        fn = direct ? pick_fast_vector_direct(lpr, ns, best_u, norm, rmode)
+                    : pick_fast_vector_staged(lpr, ns, best_u, norm, rmode);
     else
         fn = pick_exchange(lpr, ns);
     if (!fn)

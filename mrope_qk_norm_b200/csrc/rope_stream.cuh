@@ -65,7 +65,7 @@ __device__ __forceinline__ uint4 *ring_at(uint4 *ring, int stage, int k)
 }
 
 // Normalise, rotate and store the U rows of one work item from ring stage st.
-template <int LAYOUT, int LPR, int NS, int U, bool NORM, bool ROUND>
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE>
 __device__ __forceinline__ void stream_rows(
     const RopeParams &p, const Item &m, uint4 *ring, int st, const int (&vidx)[NS],
     const float2 (&C)[RowShape<LAYOUT, NS>::NQ], const float2 (&Sn)[RowShape<LAYOUT, NS>::NQ],
@@ -74,7 +74,7 @@ __device__ __forceinline__ void stream_rows(
 {
     constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
     constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
-    RotCoef<NQ, NORM && !ROUND> kc;
+    RotCoef<NQ, NORM && RMODE == kRoundNone> kc;
     make_coef(kc, C, Sn, GA, GB);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -92,7 +92,7 @@ __device__ __forceinline__ void stream_rows(
                 ss += __shfl_xor_sync(0xffffffffu, ss, off);
             r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
         }
-        norm_rotate<LAYOUT, NS, NORM, ROUND>(A, B, TL, r, kc, GA, GB, GT);
+        norm_rotate<LAYOUT, NS, NORM, RMODE>(A, B, TL, r, kc, GA, GB, GT);
         uint4 outv[NS];
         pack_row<LAYOUT, NS>(A, B, TL, outv);
         if (u < m.nh) {
@@ -108,13 +108,12 @@ template <int LAYOUT, int LPR, int NS, int U, bool NORM>
 __global__ void __launch_bounds__(kThreads)
 rope_stream_kernel(const __grid_constant__ RopeParams p)
 {
-    pdl_wait();
-    pdl_trigger();
+    pdl_enter(p.independent);
     constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
     constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
     constexpr int G = kThreads / LPR;
     const int S = p.stages;
-    const bool ROUND = p.round_norm != 0;  // uniform: both paths below are warp-uniform
+    const int rmode = p.round_norm;  // uniform: the paths below are warp-uniform
 
     extern __shared__ float4 smem[];
     uint4 *ring = reinterpret_cast<uint4 *>(smem);
@@ -225,14 +224,20 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
             unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
         }
 
-        if (ROUND)
-            stream_rows<LAYOUT, LPR, NS, U, NORM, true>(p, m, ring, st, vidx, C, Sn, GA, GB, GT);
+        if (rmode == kRoundEager)
+            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundEager>(p, m, ring, st, vidx, C, Sn, GA, GB,
+                                                               GT);
+        else if (rmode == kRoundNormalized)
+            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundNormalized>(p, m, ring, st, vidx, C, Sn,
+                                                                    GA, GB, GT);
         else
-            stream_rows<LAYOUT, LPR, NS, U, NORM, false>(p, m, ring, st, vidx, C, Sn, GA, GB, GT);
+            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundNone>(p, m, ring, st, vidx, C, Sn, GA, GB,
+                                                              GT);
     }
     cp_async_wait(0);  // nothing is left in flight (the trailing groups are empty)
     if (p.Hv > 0)
         copy_v_rows<NS, LPR>(p, tok0, ntok, vidx);
+    pdl_exit(p.independent);
 }
 
 template <int LAYOUT, int LPR, int NS, int U>

@@ -4,13 +4,15 @@
 //
 // B200 mapping.  The setup writes 2 * 4 bytes per (token, section column),
 // computing one sincosf per cell; at these sizes (8 MB for 16k tokens) it is
-// bound by launch latency and by the sincosf issue rate, not by bytes.  So
-// every warp works on its own, with no block barrier: a warp owns 8
-// consecutive tokens; lanes 0..7 derive one token's (t, h, w) each (the grid
+// bound by latency (launch, the metadata loads, sincosf's dependent chain),
+// not by bytes or issue.  So every warp works on its own, with no block
+// barrier, and keeps many independent chains in flight: a warp owns 4
+// consecutive tokens; lanes 0..3 derive one token's (t, h, w) each (the grid
 // found by shuffles over a register copy of the grid boundaries when there
-// are at most 32 grids), the positions are broadcast by shuffle, and each
-// lane owns one column of every 32 (its axis, section offset and inv_freq
-// fixed for the pass), so a warp's stores to a token row are contiguous.
+// are at most 32 grids) while the lane's inv_freq loads are in flight, the
+// positions are broadcast by shuffle, and each lane owns two columns of
+// every 64 (axis, section offset and inv_freq fixed for the pass), all four
+// tokens unrolled, so a warp's stores to a token row are contiguous.
 #include <climits>
 
 #include "qkr_internal.cuh"
@@ -19,8 +21,8 @@ namespace qkr {
 namespace {
 
 constexpr int kThreads = 256;     // debug kernels
-constexpr int kVitWarps = 4;      // warps per setup CTA
-constexpr int kVitTokPerWarp = 8; // tokens one warp writes
+constexpr int kVitWarps = 8;      // warps per setup CTA
+constexpr int kVitTokPerWarp = 4; // tokens one warp writes
 constexpr int kVitThreads = 32 * kVitWarps;
 constexpr int kTokens = kVitWarps * kVitTokPerWarp;  // tokens per setup CTA
 
@@ -89,6 +91,21 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
         return;  // warp-uniform
     const int ntok = (int)min((int64_t)kVitTokPerWarp, p.N - n0);
 
+    // This lane's columns of the first two passes (all columns when P <= 64):
+    // their axis and inv_freq do not depend on the tokens, so the inv_freq
+    // loads go out now, beside the grid metadata loads below, instead of
+    // after the positions are known.
+    const int P = p.P;
+    const int end_t = p.half[0], end_h = p.half[0] + p.half[1];
+    float f01[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int col = 32 * i + lane;
+        const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
+        const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
+        f01[i] = col < P ? __ldg(p.inv[axis] + (col - off)) : 0.f;
+    }
+
     // Lane j < ntok derives the position of token n0 + j (other lanes repeat
     // the last token, so every lane runs the same code).
     const int64_t n = n0 + min(lane, ntok - 1);
@@ -113,29 +130,42 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
         token_position(p.cu, p.grids, p.G, n, p.m, tp, hp, wp);
     }
 
-    const int P = p.P;
-    const int end_t = p.half[0], end_h = p.half[0] + p.half[1];
-    for (int c0 = 0; c0 < P; c0 += 32) {  // uniform trip count
-        // this lane's column of the pass: its axis, offset and inv_freq
-        const int col = c0 + lane;
-        const bool live = col < P;
-        const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
-        const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
-        const float f = live ? __ldg(p.inv[axis] + (col - off)) : 0.f;
-        float *cdst = p.cos_out + ((int64_t)axis * p.N + n0) * P + col;
-        float *sdst = p.sin_out + ((int64_t)axis * p.N + n0) * P + col;
-#pragma unroll 4
-        for (int j = 0; j < ntok; ++j) {  // uniform trip count
-            const int pt = __shfl_sync(0xffffffffu, tp, j);
-            const int ph = __shfl_sync(0xffffffffu, hp, j);
-            const int pw = __shfl_sync(0xffffffffu, wp, j);
-            const int pos = axis == 0 ? pt : (axis == 1 ? ph : pw);
-            const float theta = __fmul_rn((float)pos, f);
-            float sv, cv;
-            sincosf(theta, &sv, &cv);
-            if (live) {
-                __stcs(cdst + (int64_t)j * P, cv);
-                __stcs(sdst + (int64_t)j * P, sv);
+    // Two columns per lane per pass (c0 + lane, c0 + 32 + lane), every token
+    // of the warp unrolled: 2 x kVitTokPerWarp independent sincosf per lane
+    // in flight, since the kernel is bound by their dependent latency, not by
+    // bytes or issue.
+    for (int c0 = 0; c0 < P; c0 += 64) {  // uniform trip count
+        int axis[2];
+        bool live[2];
+        float f[2];
+        float *cdst[2], *sdst[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int col = c0 + 32 * i + lane;
+            live[i] = col < P;
+            axis[i] = col < end_t ? 0 : (col < end_h ? 1 : 2);
+            const int off = axis[i] == 0 ? 0 : (axis[i] == 1 ? end_t : end_h);
+            f[i] = c0 == 0 ? f01[i] : (live[i] ? __ldg(p.inv[axis[i]] + (col - off)) : 0.f);
+            cdst[i] = p.cos_out + ((int64_t)axis[i] * p.N + n0) * P + col;
+            sdst[i] = p.sin_out + ((int64_t)axis[i] * p.N + n0) * P + col;
+        }
+#pragma unroll
+        for (int j = 0; j < kVitTokPerWarp; ++j) {
+            if (j < ntok) {  // warp-uniform
+                const int pt = __shfl_sync(0xffffffffu, tp, j);
+                const int ph = __shfl_sync(0xffffffffu, hp, j);
+                const int pw = __shfl_sync(0xffffffffu, wp, j);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int pos = axis[i] == 0 ? pt : (axis[i] == 1 ? ph : pw);
+                    const float theta = __fmul_rn((float)pos, f[i]);
+                    float sv, cv;
+                    sincosf(theta, &sv, &cv);
+                    if (live[i]) {
+                        __stcs(cdst[i] + (int64_t)j * P, cv);
+                        __stcs(sdst[i] + (int64_t)j * P, sv);
+                    }
+                }
             }
         }
     }

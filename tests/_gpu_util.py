@@ -40,6 +40,31 @@ def assert_bf16_close(got: torch.Tensor, ref: np.ndarray, what: str = "") -> dic
     return {"max_abs": float(err.max()) if err.size else 0.0, "nmse": nmse}
 
 
+def assert_bf16_close_or_tie(got: torch.Tensor, ref: np.ndarray, ties: np.ndarray,
+                             what: str = "") -> dict:
+    """As assert_bf16_close, for the rounding contracts that round the
+    normalised value to bf16 before the rotation: an element may miss the
+    tolerance only where the oracle marks it as depending on a value within
+    1e-3 bf16 quanta of a rounding midpoint (there the kernel's fp32 rsqrt and
+    sum of squares may round to the other neighbour, one quantum away)."""
+    g = bf16_to_f64(got).reshape(ref.shape)
+    err = np.abs(g - ref)
+    bound = BF16_ATOL + BF16_RTOL * np.abs(ref)
+    bad = ~(err <= bound)
+    unexplained = bad & ~ties
+    if unexplained.any():
+        idx = np.argwhere(unexplained)[:5]
+        rows = ["%s: got %r ref %r" % (tuple(i), g[tuple(i)], ref[tuple(i)]) for i in idx]
+        raise AssertionError("%s: %d of %d outside |err| <= 1e-2 + 1.6e-2|ref| away from a "
+                             "rounding tie; first: %s" % (what, int(unexplained.sum()), bad.size,
+                                                          "; ".join(rows)))
+    denom = float((ref ** 2).sum())
+    nmse = float(((g - ref) ** 2).sum()) / denom if denom > 0 else 0.0
+    assert nmse < NMSE_BAR, "%s: NMSE %.3g" % (what, nmse)
+    return {"max_abs": float(err.max()) if err.size else 0.0, "nmse": nmse,
+            "tie_elements": int(ties.sum()), "outside_at_ties": int(bad.sum())}
+
+
 def assert_plane_close(got: np.ndarray, ref: np.ndarray, mask: np.ndarray, what: str = ""):
     g = got[mask].astype(np.float64)
     r = ref[mask].astype(np.float64)

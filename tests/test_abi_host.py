@@ -117,7 +117,10 @@ def test_mrope_apply_refusals(qkr):
     # unknown mode / pairing / flags
     assert _mrope(qkr, mode=9) == E
     assert _mrope(qkr, pairing=3) == E
-    assert _mrope(qkr, flags=2) == E
+    assert _mrope(qkr, flags=8) == E
+    # the rounding contracts need the norm, and only one at a time
+    assert _mrope(qkr, flags=2) == E and "normalisation" in _err(qkr)
+    assert _mrope(qkr, flags=3, gq=FAKE + (6 << 20), gk=FAKE + (7 << 20)) == E
     # empty chunk: OK, nothing enqueued
     assert _mrope(qkr, T=0) == qkr.QKR_OK
     assert qkr.last_launch()["launches"] == 0

@@ -122,3 +122,72 @@ def test_launch_record_reports_overlap():
         qkr.launch_overlap(True)
     with pytest.raises(qkr.QkrError):
         qkr._check(qkr.lib().qkr_launch_overlap(2))
+
+
+def test_independent_chunks_overlap_and_stay_ordered():
+    """QKR_FLAG_INDEPENDENT on the second chunk of a chunked step (it reads
+    and writes nothing the first chunk touches): bit-identical to the whole
+    launch, and the next step -- which reads both chunks' outputs -- sees all
+    of them.  Run as a chain of steps with no host synchronisation, with the
+    overlap switch on (the flag's early start) and off (plain order)."""
+    w = W.config4(seed=95, T=3000, Hq=8, Hkv=4)
+    s = w.streams[0]
+    q0, k0 = to_dev(s.q), to_dev(s.k)
+    pos, inv = to_dev(w.angle.positions), to_dev(w.angle.inv_freq)
+    T = q0.shape[0]
+    cut = 1111
+
+    def step(q, k, chunked):
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+        if chunked:
+            for i, (t0, t1) in enumerate(((0, cut), (cut, T))):
+                qkr.mrope_apply(q[t0:t1], k[t0:t1], qo[t0:t1], ko[t0:t1], pos, inv, w.rot,
+                                w.angle.section_mode, w.angle.sections, w.pairing,
+                                token_offset=t0, flags=qkr.FLAG_INDEPENDENT if i else 0)
+        else:
+            qkr.mrope_apply(q, k, qo, ko, pos, inv, w.rot, w.angle.section_mode,
+                            w.angle.sections, w.pairing)
+        return qo, ko
+
+    def run(chunked):
+        q, k = q0, k0
+        for _ in range(10):  # each step rotates the previous step's output again
+            q, k = step(q, k, chunked)
+        return q, k
+
+    (qa, ka), (qb, kb) = _both(lambda: run(True))
+    qr, kr = run(False)
+    torch.cuda.synchronize()
+    for q, k in ((qa, ka), (qb, kb)):
+        assert torch.equal(_bits(q), _bits(qr)) and torch.equal(_bits(k), _bits(kr))
+
+
+def test_independent_flag_on_every_kernel():
+    """The flag changes no bits on the item, streaming and exchange kernels,
+    fused and rope_set_rows calls, and combines with a rounding flag."""
+    pos = np.random.default_rng(96).integers(0, 9000, (1, 77)).astype(np.int32)
+    cases = []
+    for D, rot, pairing in ((128, 128, W.PAIRING_GPTJ), (128, 128, W.PAIRING_NEOX),
+                            (64, 20, W.PAIRING_NEOX)):
+        A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                          inv_freq=W.inv_freq(1e4, rot // 2, rot).numpy())
+        cases.append(W.random_rope_case(97 + D + rot, [77], 5, 3, D, rot, pairing, A))
+    for w in cases:
+        s = w.streams[0]
+        d = (to_dev(s.q), to_dev(s.k), to_dev(s.gamma_q), to_dev(s.gamma_k))
+        a = qkr.angle_positions(to_dev(torch.as_tensor(pos)),
+                                to_dev(torch.as_tensor(np.asarray(w.angle.inv_freq))))
+        outs = []
+        try:
+            for pipe in (1, 3):
+                qkr.tune_rope(pipe, 0, 0, 0)
+                for flags in (0, qkr.FLAG_INDEPENDENT, 2, 2 | qkr.FLAG_INDEPENDENT):
+                    qo, ko = torch.empty_like(d[0]), torch.empty_like(d[1])
+                    qkr.fused_qk_norm_rope([d], qo, ko, w.rot, w.pairing, w.eps, a, flags)
+                    outs.append((flags, qo, ko))
+        finally:
+            qkr.tune_rope(0, 0, 0, 0)
+        torch.cuda.synchronize()
+        for flags, qo, ko in outs:
+            ref = [o for o in outs if o[0] == (flags & 2)][0]
+            assert torch.equal(_bits(qo), _bits(ref[1])) and torch.equal(_bits(ko), _bits(ref[2]))

@@ -52,8 +52,39 @@ def check(w, rows=None, out_is_x=False):
 @pytest.mark.parametrize("R", [1, 32])
 def test_decode_config(R):
     info = check(W.config2(R=R, hidden=5120))
-    # a handful of rows cannot fill the GPU one CTA per row: split over a cluster
-    assert info["kernel_name"] == "rms_cluster" and info["cluster"] == (8 if R <= 8 else 4)
+    # a decode row of 5120 fits one CTA with every vector in flight at once
+    # (640 threads x one 16-byte vector of x and of the residual)
+    assert info["kernel_name"] == "rms_rows" and info["block"] == 640 and info["slots"] == 1
+
+
+@pytest.mark.parametrize("hidden", [16384, 32768, 65536])
+@pytest.mark.parametrize("R", [1, 8, 17, 32, 33])
+def test_wide_rows_split_over_a_cluster(R, hidden):
+    """Rows wider than one CTA's 1024 vectors are split over a thread-block
+    cluster at decode sizes (8 CTAs up to 16 rows, 4 up to 32); beyond that,
+    one CTA per row."""
+    info = check(W.config2(R=R, hidden=hidden, seed=700 + R))
+    if R <= 32:
+        assert info["kernel_name"] == "rms_cluster" and info["cluster"] == (8 if R <= 16 else 4)
+    else:
+        assert info["kernel_name"] == "rms_rows"
+
+
+@pytest.mark.parametrize("R,hidden", [(2, 8192), (5, 4096), (3, 65536)])
+def test_every_split_and_width(R, hidden):
+    """Every (CTAs per row, threads per CTA) choice: the residual stream is
+    bit-identical and the output within tolerance of the oracle."""
+    w = W.config2(R=R, hidden=hidden, seed=800 + R)
+    try:
+        for cs, thr in [(1, 0), (1, 256), (1, 1024), (2, 512), (4, 128), (8, 256), (16, 64),
+                        (16, 0)]:
+            if hidden // 8 // cs > 8 * (thr or 1024):
+                continue
+            qkr.tune_rms(cs, thr)
+            info = check(w)
+            assert info["cluster"] == cs
+    finally:
+        qkr.tune_rms(0, 0)
 
 
 @pytest.mark.parametrize("hidden", [2048, 4096, 8192])

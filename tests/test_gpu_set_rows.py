@@ -145,7 +145,8 @@ def test_out_of_range_row_is_skipped_and_reported():
 
 def test_scatter_full_size():
     """The measured size: 8192 tokens x 8 K heads into a 16384-row cache, in
-    the launch shape the launcher picks for it (16 tokens per CTA)."""
+    the launch shape the launcher picks for it (16 tokens per CTA, since a
+    token has only 8 heads)."""
     w = _case(W.SECTIONS_INTERLEAVED, T=8192, seed=521)
     R = 16384
     idx = np.random.default_rng(21).permutation(R)[:8192]
