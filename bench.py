@@ -274,6 +274,16 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
            [lambda s=s: s.launch(stream) for s in sets], b3, 4608, "tokens")
     del sets
 
+    # config 3 (GPT-J) with the eager-chain rounding preset, beside the default
+    # (the headline) for its cost
+    w3e = W.config3()
+    sets = [FusedSet(w3e, dev) for _ in range(n_sets_for(b3))]
+    record("fused_qk_norm_rope", "joint 512+4096 tokens H=24 D=128 GPT-J, eager rounding preset",
+           [lambda s=s: qkr.fused_qk_norm_rope(s.descs, s.qo, s.ko, 128, w3e.pairing, w3e.eps,
+                                               s.angle, qkr.FLAG_EAGER_ROUNDING, stream)
+            for s in sets], b3, 4608, "tokens", {"flags": "QKR_FLAG_EAGER_ROUNDING"})
+    del sets
+
     # config 3 as the joint Q/K/V op: V of both streams copied into the joint V
     w3 = W.config3()
     b3v = b3 + 2 * 4608 * 24 * 128 * 2
@@ -378,6 +388,14 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
             for x in s5], apply_bytes, N, "tokens", {"rotating_sets": len(s5)})
     del s5, planes
 
+    # the launch floor: an empty kernel with the library's launch attributes,
+    # back to back like every row (what a launch that moves kilobytes costs)
+    if want("launch floor"):
+        total, _ = time_launches([lambda: qkr.null_launch(1, 128, stream)], steps, warmup, stream)
+        rows.append({"kernel": "qkr_null_launch", "workload": "launch floor: empty kernel, 1 CTA",
+                     "us_per_launch": round(1e3 * total / steps, 3), "algorithmic_bytes": 0,
+                     "launch": qkr.last_launch()})
+
     # config 2: RMSNorm + residual, decode rows and sweep points
     for R, hidden in [(1, 5120), (32, 5120), (1024, 8192), (4096, 8192), (16384, 8192),
                       (16384, 2048)]:
@@ -403,6 +421,11 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
                     for s, o in zip(sets, outs8)], nb8, R, "rows")
             del outs8
         del sets
+    floor = [r["us_per_launch"] for r in rows if r["kernel"] == "qkr_null_launch"]
+    if floor:
+        for r in rows:
+            if r["kernel"].startswith("rms_norm") and r["workload"].startswith("R=1 "):
+                r["multiple_of_launch_floor"] = round(r["us_per_launch"] / floor[0], 2)
     torch.cuda.synchronize()
     return rows
 

@@ -250,6 +250,8 @@ cudaError_t launch_rms_norm_residual(const RmsParams &p, cudaStream_t stream, La
     int vpt, threads;
     const int per = (nvec + cs - 1) / cs;
     int target = cs == 8 ? 512 : (p.R <= 128 ? 1024 : (per + 1) / 2);
+    if (target > kMaxThreads)
+        target = kMaxThreads;  // wider rows take more vectors per thread
     if (target < 32)
         target = 32;
     if (g_force_threads > 0)
