@@ -30,13 +30,23 @@ KernelFn pick_stream_vector(int lpr, int ns, int u, bool norm);
 
 namespace {
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src, bool valid)
+// 16-byte copy global -> shared (shared-window address), zero-filled when
+// !valid (source size 0), so sums of squares over dead vectors stay exact.
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gmem_src, bool valid)
 {
-    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
     const int src_size = valid ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src),
-                 "r"(src_size)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_dst),
+                 "l"(gmem_src), "r"(src_size)
                  : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t smem_src)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_src)
+                 : "memory");
+    return v;
 }
 __device__ __forceinline__ void cp_async_commit()
 {
@@ -57,17 +67,19 @@ __device__ __forceinline__ void cp_async_wait(int pending)
 
 // Shared-memory ring geometry: stage s, vector k = u * NS + slot, thread t
 // at ((s * U * NS + k) * kThreads + t) * 16 bytes -- a warp's accesses to one
-// vector index are 512 consecutive bytes (conflict-free 128-bit access).
+// vector index are 512 consecutive bytes (conflict-free 128-bit access).  A
+// thread keeps the shared-window address of its stage-0 vector 0; a stage
+// adds a compile-time stride, a vector a compile-time offset.
 template <int U, int NS>
-__device__ __forceinline__ uint4 *ring_at(uint4 *ring, int stage, int k)
-{
-    return ring + ((size_t)(stage * U * NS + k) * kThreads + threadIdx.x);
-}
+struct Ring {
+    static constexpr uint32_t kVecStride = kThreads * 16;
+    static constexpr uint32_t kStageStride = U * NS * kVecStride;
+};
 
 // Normalise, rotate and store the U rows of one work item from ring stage st.
 template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE>
 __device__ __forceinline__ void stream_rows(
-    const RopeParams &p, const Item &m, uint4 *ring, int st, const int (&vidx)[NS],
+    const RopeParams &p, const Item &m, uint32_t stage_addr, const int (&vidx)[NS],
     const float2 (&C)[RowShape<LAYOUT, NS>::NQ], const float2 (&Sn)[RowShape<LAYOUT, NS>::NQ],
     const float2 (&GA)[RowShape<LAYOUT, NS>::NQ], const float2 (&GB)[RowShape<LAYOUT, NS>::NQ],
     const float2 (&GT)[RowShape<LAYOUT, NS>::NTA][4])
@@ -81,7 +93,7 @@ __device__ __forceinline__ void stream_rows(
         uint4 raw[NS];
 #pragma unroll
         for (int k = 0; k < NS; ++k)
-            raw[k] = *ring_at<U, NS>(ring, st, u * NS + k);
+            raw[k] = lds128(stage_addr + (u * NS + k) * Ring<U, NS>::kVecStride);
         float2 A[NQ], B[NQ], TL[NTA][4];
         unpack_row<LAYOUT, NS>(raw, A, B, TL);
         float r = 1.f;
@@ -152,11 +164,14 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     const int passes = (items + G - 1) / G;  // uniform across the CTA
 
     // Copy this thread's vectors of pass `pass` into ring stage `pass % S`
-    // (one commit group per pass, empty past the last pass).
+    // (one commit group per pass, empty past the last pass).  Passes are
+    // issued in order, so the stage is a counter that wraps at S.
     const int dq = G / gpt, dr = G - (G / gpt) * gpt;
     ItemCursor icur, ccur;  // the pass being copied in, the pass being computed
     icur.start(grp, gpt);
     ccur = icur;
+    const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(ring) + threadIdx.x * 16;
+    int ist = 0, cst = 0;   // ring stage being issued into, being computed from
     // With a two-pass ring the item a pass computes is the one the previous
     // issue decoded: carry it instead of decoding it again.
     Item carried;
@@ -165,16 +180,17 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
             const Item m = decode_item<U>(p, tok0, icur, ntok, nbq);
             carried = m;
             icur.advance(dq, dr, gpt);
-            const int st = pass % S;
+            const uint32_t sa = ring_base + ist * Ring<U, NS>::kStageStride;
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int k = 0; k < NS; ++k) {
                     const bool ok = u < m.nh && vidx[k] >= 0;
                     const __nv_bfloat16 *src = ok ? m.src + u * m.hs + 8 * vidx[k] : m.src;
-                    cp_async16(ring_at<U, NS>(ring, st, u * NS + k), src, ok);
+                    cp_async16(sa + (u * NS + k) * Ring<U, NS>::kVecStride, src, ok);
                 }
         }
+        ist = ist + 1 == S ? 0 : ist + 1;
         cp_async_commit();
     };
 
@@ -193,7 +209,8 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
         }
         issue(pass + S - 1);
         cp_async_wait(S - 1);
-        const int st = pass % S;
+        const uint32_t stage_addr = ring_base + cst * Ring<U, NS>::kStageStride;
+        cst = cst + 1 == S ? 0 : cst + 1;
 
         float2 C[NQ], Sn[NQ];
         {
@@ -225,13 +242,13 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
         }
 
         if (rmode == kRoundEager)
-            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundEager>(p, m, ring, st, vidx, C, Sn, GA, GB,
+            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundEager>(p, m, stage_addr, vidx, C, Sn, GA, GB,
                                                                GT);
         else if (rmode == kRoundNormalized)
-            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundNormalized>(p, m, ring, st, vidx, C, Sn,
+            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundNormalized>(p, m, stage_addr, vidx, C, Sn,
                                                                     GA, GB, GT);
         else
-            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundNone>(p, m, ring, st, vidx, C, Sn, GA, GB,
+            stream_rows<LAYOUT, LPR, NS, U, NORM, kRoundNone>(p, m, stage_addr, vidx, C, Sn, GA, GB,
                                                               GT);
     }
     cp_async_wait(0);  // nothing is left in flight (the trailing groups are empty)
