@@ -239,7 +239,10 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
     def want(workload):
         return only is None or only in workload
 
-    def record(name, workload, fns, nbytes, units, unit_name, extra=None):
+    def record(name, workload, fns, nbytes, units, unit_name, extra=None, torch_ref=None):
+        """torch_ref: (description, fns) of a torch op with the row's memory
+        traffic, timed the same way (default: the vectorised elementwise
+        kernel over the same bytes, half read and half written)."""
         if not want(workload):
             return
         total, per = time_launches(fns, steps, warmup, stream)
@@ -250,6 +253,15 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
              "frac_of_measured_hbm": round(gbs / peak_gbs, 4),
              unit_name + "_per_s": round(units / (us * 1e-6), 1),
              "launch": qkr.last_launch()}
+        if torch_ref is None:
+            ref_us = same_size_elementwise_us(nbytes, dev, stream, steps)
+            ref_what = "torch elementwise dst = -src over the same bytes"
+        else:
+            ref_what, ref_fns = torch_ref
+            ref_total, _ = time_launches(ref_fns, steps, warmup, stream)
+            ref_us = 1e3 * ref_total / steps
+        r["torch_same_traffic"] = {"op": ref_what, "us_per_launch": round(ref_us, 3),
+                                   "ratio_to_this_row": round(ref_us / us, 4)}
         if extra:
             r.update(extra)
         rows.append(r)
@@ -351,7 +363,9 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
            [lambda x=x: qkr.rope_set_rows(x[0], x[1], x[2], pos4, inv4, 128,
                                           W.SECTIONS_INTERLEAVED, (24, 20, 20), 0,
                                           stream=stream) for x in sr_sets],
-           b_sr, 8192, "tokens")
+           b_sr, 8192, "tokens",
+           torch_ref=("torch index_copy_ of the same K rows into the same cache rows",
+                      [lambda x=x: x[1].index_copy_(0, x[2], x[0]) for x in sr_sets]))
     del sr_sets
 
     # config 5: ViT setup and apply, each over rotating output/input sets
@@ -368,10 +382,14 @@ def measure_rows(dev, stream, peak_gbs, steps=200, warmup=20, only=None):
     for _ in range(n_sets_for(setup_bytes)):
         cos5 = torch.empty(3, N, 64, dtype=torch.float32, device=dev)
         planes.append((cos5, torch.empty_like(cos5)))
+    flat = [torch.empty(2 * N * 64, dtype=torch.float32, device=dev) for _ in planes]
     record("vit_mrope_setup", "8 grids N=%d, planes (3,N,64) fp32" % N,
            [lambda c=c: qkr.vit_mrope_setup(inv_t, inv_h, inv_w, cu_d, grids_d, N, 2, c[0], c[1],
                                             stream) for c in planes],
-           setup_bytes, N, "tokens", {"rotating_sets": len(planes)})
+           setup_bytes, N, "tokens", {"rotating_sets": len(planes)},
+           torch_ref=("torch fill_ of a buffer of the bytes the setup writes (write only)",
+                      [lambda f=f: f.fill_(1.0) for f in flat]))
+    del flat
     cos5, sin5 = planes[0]
     qkr.vit_mrope_setup(inv_t, inv_h, inv_w, cu_d, grids_d, N, 2, cos5, sin5, stream)
     del planes[1:]

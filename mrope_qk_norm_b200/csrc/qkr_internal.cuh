@@ -184,6 +184,8 @@ struct RopeParams {
     int Hv;                   // V heads copied into v_out (0: Q/K only)
     int rows_per_token;       // Hq + Hk + Hv
     int tokens_per_cta;
+    int tok_base, tok_rem;    // balanced split over the grid: CTA c owns tok_base tokens,
+                              // one more when c < tok_rem (T / grid, T % grid)
     int pw;                   // (cos, sin) columns staged per token: P, or D/2 for GPT-J
                               // (pairs in [P, D/2) get the identity (1, 0))
     float eps, inv_D;

@@ -58,15 +58,35 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// The CTA's range of joint tokens: CTA c owns tok_base tokens, plus one when
+// c < tok_rem (tok_base = T / grid, tok_rem = T % grid, set by the launcher),
+// so the ranges are balanced and contiguous.  T < 2^31 (checked by the
+// launcher), so 32-bit arithmetic is exact -- the 64-bit division a
+// c * T / grid split needs costs every thread ~100 instructions.
+__device__ __forceinline__ int64_t cta_first_token(const RopeParams &p)
+{
+    const int c = (int)blockIdx.x;
+    return (int64_t)(c * p.tok_base + min(c, p.tok_rem));
+}
+__device__ __forceinline__ int cta_tokens(const RopeParams &p)
+{
+    return p.tok_base + ((int)blockIdx.x < p.tok_rem ? 1 : 0);
+}
+
 // Stage (cos, sin) of `ntok` tokens into shared memory, SoA, row stride cs_ld.
-// Columns [P, pw) get the identity rotation (1, 0).
+// Columns [P, pw) get the identity rotation (1, 0).  Thread i takes cells
+// i, i + kThreads, ... of the ntok x pw tile; its (token, column) advances by
+// a fixed step instead of a division per cell.
 __device__ __forceinline__ void stage_angles(const RopeParams &p, int64_t tok0, int ntok,
                                              int cs_ld, float *cosv, float *sinv)
 {
     const int pw = p.pw;
-    for (int idx = threadIdx.x; idx < ntok * pw; idx += kThreads) {
-        const int tt = idx / pw;
-        const int j = idx - tt * pw;
+    if (pw <= 0)
+        return;
+    const int dt = kThreads / pw, dj = kThreads - (kThreads / pw) * pw;
+    int tt = (int)threadIdx.x / pw;
+    int j = (int)threadIdx.x - tt * pw;
+    while (tt < ntok) {
         float c = 1.f, s = 0.f;
         if (j < p.P) {
             const int64_t n = p.token_offset + tok0 + tt;
@@ -83,6 +103,12 @@ __device__ __forceinline__ void stage_angles(const RopeParams &p, int64_t tok0, 
         }
         cosv[tt * cs_ld + j] = c;
         sinv[tt * cs_ld + j] = s;
+        tt += dt;
+        j += dj;
+        if (j >= pw) {
+            j -= pw;
+            ++tt;
+        }
     }
 }
 
@@ -215,8 +241,7 @@ __device__ __forceinline__ void copy_v_rows(const RopeParams &p, int64_t tok0, i
 }
 
 template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE, bool DIRECT>
-__global__ void __launch_bounds__(kThreads)
-rope_fast_kernel(const __grid_constant__ RopeParams p)
+__device__ __forceinline__ void rope_fast_body(const RopeParams &p)
 {
     pdl_enter(p.independent);
     // Quads (couples of pairs) per lane: PAIRED lo/hi vectors hold 4, each
@@ -230,10 +255,9 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
     float *cosv = reinterpret_cast<float *>(smem);
     float *sinv = cosv + p.tokens_per_cta * cs_ld;
 
-    // CTA c owns joint tokens [c T / grid, (c+1) T / grid): balanced ranges of
-    // at most tokens_per_cta tokens (T < 2^31, checked by the launcher).
-    const int64_t tok0 = (int64_t)blockIdx.x * p.T / gridDim.x;
-    const int ntok = (int)((int64_t)(blockIdx.x + 1) * p.T / gridDim.x - tok0);
+    // Balanced ranges of at most tokens_per_cta consecutive joint tokens.
+    const int64_t tok0 = cta_first_token(p);
+    const int ntok = cta_tokens(p);
     if (!DIRECT) {
         stage_angles(p, tok0, ntok, cs_ld, cosv, sinv);
         __syncthreads();
@@ -349,18 +373,65 @@ rope_fast_kernel(const __grid_constant__ RopeParams p)
     pdl_exit(p.independent);
 }
 
+// The item kernel under three register policies, picked by shape, because
+// the allocation decides how many CTAs share an SM and the compiler's own
+// choice moves with small code changes:
+//   * rope_fast_kernel_narrow, one 16-byte vector per lane (GPT-J rows of
+//     up to 128 elements) without the norm or with the normalised-value
+//     rounding: at least 4 CTAs per SM (64 registers; 5 for items of at
+//     most 2 heads or without the norm).  Left to itself the compiler gave
+//     these 58-77 registers.  Items of at most 2 heads with the norm stay
+//     with the compiler: bounded to 5 CTAs they ran 5% slower (GPT-J,
+//     positions, 1024 tokens);
+//   * rope_fast_kernel_wide, NeoX rows of three or more slots (ViT apply at
+//     D=80, 4 heads per item, ~126 registers): at least 2 CTAs per SM.  A
+//     139-register build of that shape ran at one CTA per SM, 28% slower;
+//   * rope_fast_kernel, the rest: the compiler's own allocation.  On the
+//     GPT-J headline shape (4 heads per item) that is 64 registers, 4 CTAs
+//     per SM; a declared minimum of 4 CTAs gave 64 registers too but ran
+//     0.7% slower, and a minimum of 2 let it take 88 (2 CTAs per SM).
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE, bool DIRECT>
+__global__ void __launch_bounds__(kThreads) rope_fast_kernel(const __grid_constant__ RopeParams p)
+{
+    rope_fast_body<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>(p);
+}
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, 2)
+rope_fast_kernel_wide(const __grid_constant__ RopeParams p)
+{
+    rope_fast_body<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>(p);
+}
+
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE, bool DIRECT>
+__global__ void __launch_bounds__(kThreads, NORM && U > 2 ? 4 : 5)
+rope_fast_kernel_narrow(const __grid_constant__ RopeParams p)
+{
+    rope_fast_body<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>(p);
+}
+
+template <int LAYOUT, int LPR, int NS, int U, bool NORM, int RMODE, bool DIRECT>
+constexpr KernelFn item_kernel()
+{
+    if constexpr (LAYOUT == PAIRED && NS >= 3)
+        return rope_fast_kernel_wide<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>;
+    else if constexpr (LAYOUT == VECTOR && NS == 1 &&
+                       (!NORM || RMODE == kRoundNormalized))
+        return rope_fast_kernel_narrow<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>;
+    else
+        return rope_fast_kernel<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>;
+}
+
 // ------------------------------------------------------------- pickers --
 
 template <int LAYOUT, bool DIRECT, int LPR, int NS, int U>
 KernelFn pick_flags(bool norm, int rmode)
 {
     if (!norm)
-        return rope_fast_kernel<LAYOUT, LPR, NS, U, false, kRoundNone, DIRECT>;
+        return item_kernel<LAYOUT, LPR, NS, U, false, kRoundNone, DIRECT>();
     switch (rmode) {
-    case kRoundNone: return rope_fast_kernel<LAYOUT, LPR, NS, U, true, kRoundNone, DIRECT>;
-    case kRoundNormalized:
-        return rope_fast_kernel<LAYOUT, LPR, NS, U, true, kRoundNormalized, DIRECT>;
-    case kRoundEager: return rope_fast_kernel<LAYOUT, LPR, NS, U, true, kRoundEager, DIRECT>;
+    case kRoundNone: return item_kernel<LAYOUT, LPR, NS, U, true, kRoundNone, DIRECT>();
+    case kRoundNormalized: return item_kernel<LAYOUT, LPR, NS, U, true, kRoundNormalized, DIRECT>();
+    case kRoundEager: return item_kernel<LAYOUT, LPR, NS, U, true, kRoundEager, DIRECT>();
     default: return nullptr;
     }
 }

@@ -314,6 +314,8 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
     if (grid < 1)
         grid = 1;
     p.tokens_per_cta = (int)((p.T + grid - 1) / grid);
+    p.tok_base = (int)(p.T / grid);
+    p.tok_rem = (int)(p.T % grid);
     const size_t smem = ring + (size_t)p.tokens_per_cta * cs_ld * 2 * sizeof(float);
     e = launch(fn, dim3((unsigned)grid), dim3(kThreads), smem, stream, 1, p);
     if (e == cudaSuccess && rec) {
@@ -482,6 +484,8 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
         grid = 1;
     // the exchange kernel walks fixed tiles; the item kernels take balanced ranges
     p.tokens_per_cta = (int)((p.T + grid - 1) / grid);
+    p.tok_base = (int)(p.T / grid);
+    p.tok_rem = (int)(p.T % grid);
 
     size_t smem = staged ? (size_t)p.tokens_per_cta * cs_ld * 2 * sizeof(float) : 0;
     if (layout == EXCHANGE)

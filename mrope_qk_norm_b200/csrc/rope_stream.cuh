@@ -133,8 +133,8 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     float *cosv = reinterpret_cast<float *>(ring + (size_t)S * U * NS * kThreads);
     float *sinv = cosv + p.tokens_per_cta * cs_ld;
 
-    const int64_t tok0 = (int64_t)blockIdx.x * p.T / gridDim.x;
-    const int ntok = (int)((int64_t)(blockIdx.x + 1) * p.T / gridDim.x - tok0);
+    const int64_t tok0 = cta_first_token(p);
+    const int ntok = cta_tokens(p);
 
     const int lane = threadIdx.x % LPR;
     const int grp = threadIdx.x / LPR;

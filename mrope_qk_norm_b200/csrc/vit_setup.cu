@@ -132,10 +132,73 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
         token_position(p.cu, p.grids, p.G, n, p.m, tp, hp, wp);
     }
 
-    // Two columns per lane per pass (c0 + lane, c0 + 32 + lane), every token
-    // of the warp unrolled: 2 x kVitTokPerWarp independent sincosf per lane
-    // in flight, since the kernel is bound by their dependent latency, not by
-    // bytes or issue.
+    // Merge size 2 with h and w even (every grid then starts on a multiple
+    // of 4 tokens): the warp's 8 tokens are two whole 2x2 merge blocks, token
+    // 4b + 2i + k at (t_b, h_b + i, w_b + k) from its block's first patch.  A
+    // column then takes at most 4 distinct angles over the 8 tokens (t: one
+    // per block, h: h_b + {0, 1}, w: w_b + {0, 1}), so each lane computes 4
+    // sincosf per column instead of 8 and picks per token.  The same
+    // expression on the same position, so the values are identical.  The
+    // warp checks the pattern on its own positions and otherwise takes the
+    // general loop below.
+    const int bt0 = __shfl_sync(0xffffffffu, tp, 0), bt1 = __shfl_sync(0xffffffffu, tp, 4);
+    const int bh0 = __shfl_sync(0xffffffffu, hp, 0), bh1 = __shfl_sync(0xffffffffu, hp, 4);
+    const int bw0 = __shfl_sync(0xffffffffu, wp, 0), bw1 = __shfl_sync(0xffffffffu, wp, 4);
+    bool blocks = false;
+    if (p.m == 2 && ntok == kVitTokPerWarp) {  // warp-uniform
+        const int b = (lane >> 2) & 1;
+        const bool ok = lane >= kVitTokPerWarp ||
+                        (tp == (b ? bt1 : bt0) && hp == (b ? bh1 : bh0) + ((lane >> 1) & 1) &&
+                         wp == (b ? bw1 : bw0) + (lane & 1));
+        blocks = __all_sync(0xffffffffu, ok);
+    }
+    if (blocks) {
+        for (int c0 = 0; c0 < P; c0 += 64) {  // uniform trip count
+            int axis[2];
+            bool live[2];
+            float *cdst[2], *sdst[2];
+            float cv[2][4], sv[2][4];  // slot s = 2b + d: block b, offset d on h / w
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int col = c0 + 32 * i + lane;
+                live[i] = col < P;
+                axis[i] = col < end_t ? 0 : (col < end_h ? 1 : 2);
+                const int off = axis[i] == 0 ? 0 : (axis[i] == 1 ? end_t : end_h);
+                const float f =
+                    c0 == 0 ? f01[i] : (live[i] ? __ldg(p.inv[axis[i]] + (col - off)) : 0.f);
+                cdst[i] = p.cos_out + ((int64_t)axis[i] * p.N + n0) * P + col;
+                sdst[i] = p.sin_out + ((int64_t)axis[i] * p.N + n0) * P + col;
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    const int d = sl & 1;
+                    const int pos = axis[i] == 0   ? (sl < 2 ? bt0 : bt1)
+                                    : axis[i] == 1 ? (sl < 2 ? bh0 : bh1) + d
+                                                   : (sl < 2 ? bw0 : bw1) + d;
+                    sincosf(__fmul_rn((float)pos, f), &sv[i][sl], &cv[i][sl]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kVitTokPerWarp; ++j) {
+                const int st = 2 * (j >> 2), sh = st + ((j >> 1) & 1), sw = st + (j & 1);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    // st, sh, sw are constants once unrolled: register picks
+                    const float c = axis[i] == 0 ? cv[i][st] : (axis[i] == 1 ? cv[i][sh] : cv[i][sw]);
+                    const float sn = axis[i] == 0 ? sv[i][st] : (axis[i] == 1 ? sv[i][sh] : sv[i][sw]);
+                    if (live[i]) {
+                        __stcs(cdst[i] + (int64_t)j * P, c);
+                        __stcs(sdst[i] + (int64_t)j * P, sn);
+                    }
+                }
+            }
+        }
+        return;
+    }
+
+    // General case.  Two columns per lane per pass (c0 + lane, c0 + 32 +
+    // lane), every token of the warp unrolled: 2 x kVitTokPerWarp independent
+    // sincosf per lane in flight, since the kernel is bound by their dependent
+    // latency, not by bytes or issue.
     for (int c0 = 0; c0 < P; c0 += 64) {  // uniform trip count
         int axis[2];
         bool live[2];

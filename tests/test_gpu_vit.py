@@ -95,12 +95,15 @@ def test_setup_many_grids_and_long_axis():
     assert np.array_equal(cos.untouched(), ~mask)
 
 
-@pytest.mark.parametrize("lens,m", [((64, 64, 64), 1), ((4, 6, 6), 1), ((16, 24, 24), 4)])
+@pytest.mark.parametrize("lens,m", [((64, 64, 64), 1), ((4, 6, 6), 1), ((16, 24, 24), 4),
+                                    ((16, 24, 24), 2), ((3, 5, 7), 2)])
 def test_setup_empty_grids_and_narrow_grids(lens, m):
     """Grids with zero frames among at most 32 grids (the kernel finds a
-    token's grid by shuffles over the boundaries), merge sizes 1 and 4, and
-    grids one merge block wide (8 consecutive tokens of a warp then span 8
-    h positions): planes and positions equal the oracle's."""
+    token's grid by shuffles over the boundaries), merge sizes 1, 2 and 4,
+    and grids one merge block wide (8 consecutive tokens of a warp then span
+    8 h positions; at merge size 2, two merge blocks in different block
+    rows, which the kernel's two-block path handles): planes and positions
+    equal the oracle's."""
     grids = [[1, 8 * m, m], [0, 4 * m, 4 * m], [2, 2 * m, 6 * m], [0, m, m], [1, 16 * m, m],
              [1, 4 * m, 4 * m]]
     w = W.config5(seed=57, grids=grids, lens=lens, spatial_merge=m)
