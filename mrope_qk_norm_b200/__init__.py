@@ -168,7 +168,8 @@ def _ptr_base(t, dtype, what):
 def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 0,
               stages: int = 0) -> None:
     """Override the rope kernels' launch shape (0 = automatic), for tuning.
-    pipeline: 1 item kernel, 2 bulk-copy pipelined kernel, 3 streaming kernel."""
+    pipeline: 1 item kernel, 3 streaming kernel; stages: depth of the
+    streaming kernel's row ring (0 automatic, 1 and 2 both mean 2, up to 4)."""
     _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta, stages))
 
 

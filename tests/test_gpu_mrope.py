@@ -179,3 +179,37 @@ def test_packed_qkv_in_place():
     assert torch.equal(qv.view(torch.int16), ref_q.view(torch.int16))
     assert torch.equal(kv.view(torch.int16), ref_k.view(torch.int16))
     assert torch.equal(buf[:, 2].view(torch.int16), v_before.view(torch.int16))
+
+
+@pytest.mark.parametrize("pipeline", [0, 1, 3])
+def test_row_offsets_past_2_31(pipeline):
+    """Row offsets the kernel forms past 2^31 elements on the positions path:
+    Q is a view whose token stride puts token 2 beyond 2^31 elements from its
+    base.  Item kernel and streaming kernel alike equal the contiguous launch
+    bit for bit.  About 4.3 GiB for the wide view."""
+    free, _ = torch.cuda.mem_get_info()
+    if free < 8 * 2 ** 30:
+        pytest.skip("needs 8 GiB of free device memory")
+    w = W.config4(seed=93, T=3, Hq=2, Hkv=1)
+    q, k, pos, inv = _dev_inputs(w)
+    T, Hq, D = q.shape
+    ts = 2 ** 30 + 8
+    assert (T - 1) * ts > 2 ** 31
+    big = torch.empty((T - 1) * ts + Hq * D, dtype=torch.bfloat16, device="cuda")
+    qw = big.as_strided((T, Hq, D), (ts, D, 1))
+    qw.copy_(q)
+    try:
+        qkr.tune_rope(pipeline, 0, 0, 0)
+        ref_q, ref_k = run_mrope(w)
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+        qkr.mrope_apply(qw, k, qo, ko, pos, inv, w.rot, w.angle.section_mode, w.angle.sections,
+                        w.pairing)
+        torch.cuda.synchronize()
+        name = qkr.last_launch()["kernel_name"]
+    finally:
+        qkr.tune_rope(0, 0, 0, 0)
+    assert name == "rope_paired"
+    assert torch.equal(qo.view(torch.int16), ref_q.view(torch.int16))
+    assert torch.equal(ko.view(torch.int16), ref_k.view(torch.int16))
+    del big, qw
+    torch.cuda.empty_cache()
