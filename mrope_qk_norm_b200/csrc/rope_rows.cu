@@ -283,15 +283,16 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
     cudaError_t e = allow_smem(fn, ring + angles_max);
     if (e != cudaSuccess)
         return e;
-    // Token split: 8 tokens per CTA once that still fills a wave of resident
-    // CTAs, else 4.  On interleaved mRoPE (8192 x (16+8) heads) launches of
-    // 8192 and 5735 tokens were fastest at 8 and one of 2457 at 4 (8.5 us
-    // against 9.3 us at 8, whose grid is half a wave); 16 tokens per CTA
-    // was 8-13% slower on all three (each CTA's staging prologue is exposed
-    // once per range, over fewer CTAs).  Whole waves of balanced ranges
-    // (grid a multiple of the resident CTAs, at most 8 tokens each) were
-    // slower still: the chunked pair took 24.35 us against 23.96 us, more
-    // CTAs paying the prologue costing more than the partly filled last wave.
+    // Token split: the fewest whole waves of resident CTAs at no more than 7
+    // tokens per CTA, tokens shared out evenly (at least 4 per CTA).  A sweep
+    // of interleaved mRoPE launches (16+8 heads, T = 2400 .. 8192, 4 .. 16
+    // tokens per CTA) put the best split there: a partly filled last wave
+    // costs most (2400 tokens: 6.5 us at 5 per CTA, one wave, against 7.6 us
+    // at 4, 1.01 waves; 5000: 12.1 us at 5, two waves, against 13.2 at 8),
+    // and more than about 8 tokens per CTA exposes each CTA's staging
+    // prologue (8192: 17.5 us at 7 against 20.2 at 12).  Against the
+    // previous rule (4 per CTA below 8 x the resident CTAs, else 8) only
+    // 6000 and 7000 tokens lost, 2-4%.
     int64_t grid;
     int tt = g_force_tt;
     if (tt <= 0) {
@@ -299,14 +300,20 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
         e = resident_slots(fn, ring + (size_t)8 * cs_ld * 2 * sizeof(float), &slots);
         if (e != cudaSuccess)
             return e;
-        tt = p.T >= 8 * (int64_t)slots ? 8 : 4;
+        const int64_t waves = (p.T + 7 * (int64_t)slots - 1) / (7 * (int64_t)slots);
+        const int64_t even = (p.T + waves * slots - 1) / (waves * slots);
+        tt = even < 4 ? 4 : (int)even;
         // Few heads per token (K-only scatter into a cache: 8 heads, 4
         // items per token) would leave one item per lane group at 8
-        // tokens, so nothing overlaps the ring's first wait; 16 tokens
-        // measured 5% faster on 8192 x 8 heads of K.
+        // tokens, so nothing overlaps the ring's first wait: up to 16
+        // tokens per CTA (5% faster than 8 on 8192 x 8 heads of K), but no
+        // more than fill one wave (14 there: 586 CTAs of 592 slots, 0.8%
+        // faster than 16; 12 or 13 spill into a second wave, 20% slower).
         const int items_per_token = (p.Hq + u - 1) / u + (p.Hk + u - 1) / u;
-        if (tt == 8 && 8 * items_per_token < 2 * (kThreads / lpr))
-            tt = 16;
+        if (8 * items_per_token < 2 * (kThreads / lpr)) {
+            const int64_t wave = (p.T + slots - 1) / slots;
+            tt = wave < 8 ? 8 : (wave > 16 ? 16 : (int)wave);
+        }
     }
     if (tt > kStreamTokens)
         tt = kStreamTokens;

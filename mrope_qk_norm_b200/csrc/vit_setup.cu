@@ -28,6 +28,19 @@ constexpr int kVitTokPerWarp = 8; // tokens one warp writes
 constexpr int kVitThreads = 32 * kVitWarps;
 constexpr int kTokens = kVitWarps * kVitTokPerWarp;  // tokens per setup CTA
 
+// a / d for a, d < 2^20 (d >= 1): a single-precision quotient estimate (the
+// approximate divide is within 2 ulp, so the estimate is within 1 of a / d)
+// truncated, then made exact by one integer correction step on the
+// remainder.  Several times shorter in latency than the 32-bit integer
+// division routine, and the positions sit on the setup's critical path.
+__device__ __forceinline__ uint32_t udiv_small(uint32_t a, uint32_t d)
+{
+    uint32_t q = (uint32_t)__fdividef((float)a, (float)d);
+    const int r = (int)(a - q * d);
+    q = r < 0 ? q - 1 : (r >= (int)d ? q + 1 : q);
+    return q;
+}
+
 // (t, h, w) of the token at `local` index inside a grid of [., h, w] with
 // merge size m.  Inside a frame of h*w tokens, tokens come in m x m merge
 // blocks in row-major block order, each block's patches in row-major order.
@@ -35,9 +48,24 @@ __device__ __forceinline__ void grid_position(int64_t local, int h, int w, int m
                                               int &hp, int &wp)
 {
     const int64_t frame = max((int64_t)h * w, (int64_t)1);
+    if (local >= 0 && local < (1 << 20) && frame < (1 << 20) && m > 0 && m < 1024) {
+        // the usual case: every quotient by the short division above
+        const uint32_t l32 = (uint32_t)local, f32 = (uint32_t)frame, mm = (uint32_t)(m * m);
+        const uint32_t t32 = udiv_small(l32, f32);
+        const uint32_t in_frame = l32 - t32 * f32;
+        const uint32_t block = udiv_small(in_frame, mm);
+        const uint32_t patch = in_frame - block * mm;
+        const uint32_t bpr = (uint32_t)max(w / m, 1);
+        const uint32_t brow = udiv_small(block, bpr);
+        const uint32_t bcol = block - brow * bpr;
+        const uint32_t prow = udiv_small(patch, (uint32_t)m);
+        tp = (int)t32;
+        hp = (int)(brow * (uint32_t)m + prow);
+        wp = (int)(bcol * (uint32_t)m + (patch - prow * (uint32_t)m));
+        return;
+    }
     if (frame <= 0xffffffffLL && local >= 0 && local <= 0xffffffffLL && m > 0) {
-        // the usual case, in 32-bit unsigned arithmetic (a 64-bit division is
-        // several times longer)
+        // 32-bit unsigned arithmetic (a 64-bit division is several times longer)
         const uint32_t l32 = (uint32_t)local, f32 = (uint32_t)frame, mm = (uint32_t)(m * m);
         const uint32_t t32 = l32 / f32;
         const uint32_t in_frame = l32 - t32 * f32;
@@ -114,15 +142,21 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
     int tp, hp, wp;
     if (p.G <= 32) {
         // lane l holds grid l's boundaries and sizes: one load each, and the
-        // grid of a token is the number of grids that end at or before it
+        // grid of a token is the number of grids that end at or before it --
+        // one ballot per token of the warp (the tokens are consecutive)
         const bool have = lane < p.G;
         const int32_t end_l = have ? __ldg(p.cu + lane + 1) : 0;
         const int32_t start_l = have ? __ldg(p.cu + lane) : 0;
         const int32_t h_l = have ? __ldg(p.grids + 3 * lane + 1) : 1;
         const int32_t w_l = have ? __ldg(p.grids + 3 * lane + 2) : 1;
+        const int myj = min(lane, ntok - 1);
         int g = 0;
-        for (int k = 0; k < p.G; ++k)  // uniform trip count
-            g += (int64_t)__shfl_sync(0xffffffffu, end_l, k) <= n ? 1 : 0;
+#pragma unroll
+        for (int j = 0; j < kVitTokPerWarp; ++j) {
+            const unsigned ends = __ballot_sync(0xffffffffu, have && (int64_t)end_l <= n0 + j);
+            if (myj == j)
+                g = __popc(ends);
+        }
         g = min(g, p.G - 1);
         const int32_t start = __shfl_sync(0xffffffffu, start_l, g);
         const int32_t h = __shfl_sync(0xffffffffu, h_l, g);

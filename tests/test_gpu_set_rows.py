@@ -145,14 +145,16 @@ def test_out_of_range_row_is_skipped_and_reported():
 
 def test_scatter_full_size():
     """The measured size: 8192 tokens x 8 K heads into a 16384-row cache, in
-    the launch shape the launcher picks for it (16 tokens per CTA, since a
-    token has only 8 heads)."""
+    the launch shape the launcher picks for it (more than 8 tokens per CTA,
+    since a token has only 8 heads, and at most one wave: 14 on 148 SMs)."""
     w = _case(W.SECTIONS_INTERLEAVED, T=8192, seed=521)
     R = 16384
     idx = np.random.default_rng(21).permutation(R)[:8192]
     cache = _scatter(w, idx, R)
     rec = qkr.last_launch()
-    assert rec["pipelined"] == 2 and rec["tokens_per_cta"] == 16, rec
+    assert rec["pipelined"] == 2 and 8 < rec["tokens_per_cta"] <= 16, rec
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert rec["grid"] <= 4 * sms, rec
     rid = torch.as_tensor(idx, dtype=torch.int64, device="cuda")
     assert torch.equal(_bits(cache.tensor[rid]), _bits(_mrope_k(w))), "scatter != mrope_apply"
     assert cache.untouched()[np.setdiff1d(np.arange(R), idx)].all()

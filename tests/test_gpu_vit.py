@@ -52,6 +52,21 @@ def test_positions_bit_exact(m):
     assert np.array_equal(out.cpu().numpy(), oracle.vit_positions(grids, m))
 
 
+@pytest.mark.parametrize("m,grids", [(2, [[3, 512, 512], [1, 1024, 1024], [2, 6, 10]]),
+                                     (4, [[5, 200, 300], [1, 4, 4]]),
+                                     (1, [[2, 1023, 1025], [7, 3, 5]])])
+def test_positions_large_grids_bit_exact(m, grids):
+    """Frames and token indices on both sides of 2^20, where the kernels'
+    position derivation switches from its short single-precision division
+    (exact below 2^20) to integer division: every position equals the
+    oracle's."""
+    cu, dgrids, N = vit_meta(grids)
+    out = torch.empty(3, N, dtype=torch.int32, device="cuda")
+    qkr.vit_positions(cu, dgrids, N, m, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), oracle.vit_positions(grids, m))
+
+
 def test_setup_config_planes():
     w = W.config5()
     cos, sin, _, _, N = run_setup(w)
