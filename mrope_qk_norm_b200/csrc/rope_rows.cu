@@ -478,11 +478,39 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
         const int tt = ftt < max_tt_smem ? ftt : max_tt_smem;
         grid = (p.T + tt - 1) / tt;
     } else if (direct) {
+        // Tokens per CTA: a multiple of the count that gives every lane group
+        // the same number of work items (whole passes), the smallest whose
+        // grid fits in two waves of resident CTAs for one-vector GPT-J rows
+        // and in one wave otherwise.  Joint 512+4096 tokens x 24 heads:
+        // GPT-J at 4 per CTA (1152 CTAs, 3 passes per group) 19.95 us
+        // against 20.6 us for one balanced wave of 7-8 (6 passes, the last a
+        // quarter full on the CTAs with 7) and 20.57 at 8 per CTA (one wave,
+        // whole passes); NeoX at 16 per CTA (288 CTAs, 6 passes) 21.03 us
+        // against 21.2 at 15-16 and 21.44 at 8 (two waves).  ViT apply lost
+        // 8% on two waves.
         int slots = 0;
         cudaError_t e = resident_slots(fn, 0, &slots);
         if (e != cudaSuccess)
             return e;
-        grid = p.T < slots ? p.T : slots;
+        const int groups = kThreads / lpr;
+        const int items = (p.Hq + best_u - 1) / best_u + (p.Hk + best_u - 1) / best_u;
+        int a = items, b = groups;
+        while (b) {
+            const int r = a % b;
+            a = b;
+            b = r;
+        }
+        const int64_t unit = groups / (a > 0 ? a : 1);  // tokens per CTA for whole passes
+        const int64_t waves = layout == VECTOR && ns == 1 ? 2 : 1;
+        const int64_t cap = waves * slots;
+        int64_t tt = unit;
+        if ((p.T + tt - 1) / tt > cap)
+            tt = ((p.T + cap - 1) / cap + unit - 1) / unit * unit;
+        grid = (p.T + tt - 1) / tt;
+        // launches of fewer tokens than resident CTAs: one token per CTA
+        // spreads them over the most SMs
+        if (p.T < slots)
+            grid = p.T;
     } else {
         const int tt = 4 < max_tt_smem ? 4 : max_tt_smem;
         grid = (p.T + tt - 1) / tt;
