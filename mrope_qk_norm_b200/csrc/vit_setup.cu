@@ -109,6 +109,9 @@ __device__ __forceinline__ void token_position(const int32_t *cu, const int32_t 
                   m, tp, hp, wp);
 }
 
+// CS: columns per lane per pass of 32 * CS columns -- 2, or 1 when a row has
+// at most 32 columns (two per lane would leave the second half dead).
+template <int CS>
 __global__ void __launch_bounds__(kVitThreads)
 vit_setup_kernel(const __grid_constant__ VitParams p)
 {
@@ -117,19 +120,20 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t n0 = ((int64_t)blockIdx.x * kVitWarps + warp) * kVitTokPerWarp;
+    constexpr int cstep = 32 * CS;  // columns per pass
     if (n0 >= p.N)
         return;  // warp-uniform
     const int ntok = (int)min((int64_t)kVitTokPerWarp, p.N - n0);
 
-    // This lane's columns of the first two passes (all columns when P <= 64):
+    // This lane's columns of the first pass (all of them when P <= cstep):
     // their axis and inv_freq do not depend on the tokens, so the inv_freq
     // loads go out now, beside the grid metadata loads below, instead of
     // after the positions are known.
     const int P = p.P;
     const int end_t = p.half[0], end_h = p.half[0] + p.half[1];
-    float f01[2];
+    float f01[CS];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < CS; ++i) {
         const int col = 32 * i + lane;
         const int axis = col < end_t ? 0 : (col < end_h ? 1 : 2);
         const int off = axis == 0 ? 0 : (axis == 1 ? end_t : end_h);
@@ -187,13 +191,13 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
         blocks = __all_sync(0xffffffffu, ok);
     }
     if (blocks) {
-        for (int c0 = 0; c0 < P; c0 += 64) {  // uniform trip count
-            int axis[2];
-            bool live[2];
-            float *cdst[2], *sdst[2];
-            float cv[2][4], sv[2][4];  // slot s = 2b + d: block b, offset d on h / w
+        for (int c0 = 0; c0 < P; c0 += cstep) {  // uniform trip count
+            int axis[CS];
+            bool live[CS];
+            float *cdst[CS], *sdst[CS];
+            float cv[CS][4], sv[CS][4];  // slot s = 2b + d: block b, offset d on h / w
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < CS; ++i) {
                 const int col = c0 + 32 * i + lane;
                 live[i] = col < P;
                 axis[i] = col < end_t ? 0 : (col < end_h ? 1 : 2);
@@ -215,7 +219,7 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
             for (int j = 0; j < kVitTokPerWarp; ++j) {
                 const int st = 2 * (j >> 2), sh = st + ((j >> 1) & 1), sw = st + (j & 1);
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < CS; ++i) {
                     // st, sh, sw are constants once unrolled: register picks
                     const float c = axis[i] == 0 ? cv[i][st] : (axis[i] == 1 ? cv[i][sh] : cv[i][sw]);
                     const float sn = axis[i] == 0 ? sv[i][st] : (axis[i] == 1 ? sv[i][sh] : sv[i][sw]);
@@ -229,17 +233,17 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
         return;
     }
 
-    // General case.  Two columns per lane per pass (c0 + lane, c0 + 32 +
-    // lane), every token of the warp unrolled: 2 x kVitTokPerWarp independent
-    // sincosf per lane in flight, since the kernel is bound by their dependent
-    // latency, not by bytes or issue.
-    for (int c0 = 0; c0 < P; c0 += 64) {  // uniform trip count
-        int axis[2];
-        bool live[2];
-        float f[2];
-        float *cdst[2], *sdst[2];
+    // General case.  CS columns per lane per pass, every token of the warp
+    // unrolled: CS x kVitTokPerWarp independent sincosf per lane in flight,
+    // since the kernel is bound by their dependent latency, not by bytes or
+    // issue.
+    for (int c0 = 0; c0 < P; c0 += cstep) {  // uniform trip count
+        int axis[CS];
+        bool live[CS];
+        float f[CS];
+        float *cdst[CS], *sdst[CS];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < CS; ++i) {
             const int col = c0 + 32 * i + lane;
             live[i] = col < P;
             axis[i] = col < end_t ? 0 : (col < end_h ? 1 : 2);
@@ -255,7 +259,7 @@ vit_setup_kernel(const __grid_constant__ VitParams p)
                 const int ph = __shfl_sync(0xffffffffu, hp, j);
                 const int pw = __shfl_sync(0xffffffffu, wp, j);
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < CS; ++i) {
                     const int pos = axis[i] == 0 ? pt : (axis[i] == 1 ? ph : pw);
                     const float theta = __fmul_rn((float)pos, f[i]);
                     float sv, cv;
@@ -301,17 +305,24 @@ __global__ void section_map_kernel(const __grid_constant__ SectionArgs a, int8_t
 
 }  // namespace
 
-cudaError_t launch_vit_setup(const VitParams &p, cudaStream_t stream, LaunchRecord *rec)
+cudaError_t launch_vit_setup(const VitParams &p_in, cudaStream_t stream, LaunchRecord *rec)
 {
-    const int64_t grid = (p.N + kTokens - 1) / kTokens;
+    // Two columns per lane; one when a row has at most 32.  Splitting a
+    // block of 8 tokens' 64 columns over two warps (twice the resident warps)
+    // measured 4.17 us against 3.97 us: each warp then derives the positions.
+    const VitParams &p = p_in;
+    const int tokens = kTokens;
+    const int64_t grid = (p.N + tokens - 1) / tokens;
     if (grid > INT_MAX)
         return cudaErrorInvalidConfiguration;
-    cudaError_t err = launch(vit_setup_kernel, dim3((unsigned)grid), dim3(kVitThreads), 0,
-                             stream, 1, p);
+    cudaError_t err = p.P > 32 ? launch(vit_setup_kernel<2>, dim3((unsigned)grid),
+                                        dim3(kVitThreads), 0, stream, 1, p)
+                               : launch(vit_setup_kernel<1>, dim3((unsigned)grid),
+                                        dim3(kVitThreads), 0, stream, 1, p);
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();
         rec->kernel = QKR_KERNEL_VIT_SETUP;
-        rec->tokens_per_cta = kTokens;
+        rec->tokens_per_cta = tokens;
         rec->block = kVitThreads;
         rec->grid = grid;
         rec->launches = 1;
