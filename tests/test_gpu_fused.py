@@ -518,3 +518,18 @@ def test_streaming_kernel_shapes_and_round_flag():
     (qb, kb), _ = _with_shape(w, 1, flags=flags)
     assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
     assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+
+
+@pytest.mark.parametrize("pairing", [W.PAIRING_GPTJ, W.PAIRING_NEOX])
+@pytest.mark.parametrize("t_txt,img_h,img_w", [(77, 30, 21), (513, 64, 64)])
+def test_joint_ragged_token_counts(pairing, t_txt, img_h, img_w):
+    """Joint launches whose token count is not a multiple of the tokens per
+    CTA the direct-angle launcher picks (whole passes per lane group: 4 for
+    GPT-J, 16 for NeoX at 24 heads), so the balanced ranges differ by one
+    token across CTAs: equal to the oracle, and every token written once."""
+    w = W.config3(seed=81, T_txt=t_txt, img_h=img_h, img_w=img_w, pairing=pairing)
+    check_against_oracle(w, what="ragged joint")
+    rec = qkr.last_launch()
+    assert rec["direct_angles"] == 1
+    assert rec["grid"] * rec["tokens_per_cta"] >= w.n_tokens
+    assert (rec["grid"] - 1) * rec["tokens_per_cta"] < w.n_tokens

@@ -63,7 +63,7 @@ def test_config_full_size(mode):
     assert torch.equal(k.view(torch.int16), kc.view(torch.int16))
 
 
-@pytest.mark.parametrize("T", [2, 300, 2457, 8192])
+@pytest.mark.parametrize("T", [2, 300, 2457, 4000, 5735, 8192])
 def test_chunk_token_counts(T):
     # the token counts of the fork's known-answer cases; random chunk splits
     w = W.config4(seed=40 + T, T=T, Hq=4, Hkv=2)
