@@ -161,3 +161,22 @@ def test_scatter_full_size():
     _, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle,
                                 norm=False)
     assert_bf16_close(cache.tensor[rid], rk, "full-size scatter")
+
+
+@pytest.mark.parametrize("hk", [1, 2, 3, 8])
+def test_scatter_every_kernel_agrees(hk):
+    """The automatic choice, the item kernel with staged angles and the
+    streaming kernel give the same bits for a K-only scatter of 1..8 heads
+    (3 leaves one head of the last item dead)."""
+    w = _case(W.SECTIONS_INTERLEAVED, T=1000, seed=600 + hk, H=hk)
+    R = 1500
+    idx = np.random.default_rng(hk).permutation(R)[:1000]
+    outs = []
+    try:
+        for pipe in (0, 1, 3):
+            qkr.tune_rope(pipe, 0, 0, 0)
+            outs.append((_scatter(w, idx, R).tensor.clone(), qkr.last_launch()))
+    finally:
+        qkr.tune_rope(0, 0, 0, 0)
+    for c, rec in outs[1:]:
+        assert torch.equal(_bits(c), _bits(outs[0][0])), rec
