@@ -1,8 +1,8 @@
 // rope_math.cuh -- the per-row arithmetic shared by every lane-group rope
-// kernel (item, streaming and bulk-copy pipelined): unpacking a lane's 16-byte
-// vectors of a head row into packed fp32x2 couples, the row's sum of squares,
-// normalisation and rotation, and packing back to bf16.  Keeping one copy of it
-// is what makes the kernels bit-identical to one another.
+// kernel (item and streaming): unpacking a lane's 16-byte vectors of a head
+// row into packed fp32x2 couples, the row's sum of squares, normalisation and
+// rotation, and packing back to bf16.  Keeping one copy of it is what makes
+// the kernels bit-identical to one another.
 //
 // Couples.  A lane holds NQ "quads" of a head row, each quad two rotation
 // pairs: A = the first members of the two pairs, B = the second members, as

@@ -207,7 +207,7 @@ def test_launch_switch_refusals(qkr):
     assert L.qkr_launch_overlap(2) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_launch_overlap(-1) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(4, 0, 0, 0) == qkr.QKR_ERR_INVALID_ARG
-    assert L.qkr_tune_rope(2, 0, 0, 0) == qkr.QKR_ERR_INVALID_ARG   # no bulk-copy kernel
+    assert L.qkr_tune_rope(2, 0, 0, 0) == qkr.QKR_ERR_INVALID_ARG   # 1 item, 3 streaming only
     assert L.qkr_tune_rope(3, 0, 0, 5) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(1, 0, 0, -1) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(3, 5, 0, 0) == qkr.QKR_ERR_INVALID_ARG
