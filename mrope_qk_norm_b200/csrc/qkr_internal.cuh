@@ -186,6 +186,7 @@ struct RopeParams {
     int tokens_per_cta;
     int tok_base, tok_rem;    // balanced split over the grid: CTA c owns tok_base tokens,
                               // one more when c < tok_rem (T / grid, T % grid)
+    int gpt_recip;            // 2^16 / (work items per token), for the item cursor
     int pw;                   // (cos, sin) columns staged per token: P, or D/2 for GPT-J
                               // (pairs in [P, D/2) get the identity (1, 0))
     float eps, inv_D;

@@ -143,15 +143,27 @@ struct Item {
     bool s1;                   // second stream
 };
 
+// n / d and n % d for 0 <= n <= 256 and d >= 1, with recip = floor(2^16 / d)
+// from the host: (n * recip) >> 16 is the quotient or one short of it (the
+// error of recip is under n / 2^16 < 1), and one correction step fixes it.
+__device__ __forceinline__ void divmod_small(int n, int d, int recip, int &q, int &r)
+{
+    q = (n * recip) >> 16;
+    r = n - q * d;
+    if (r >= d) {
+        r -= d;
+        ++q;
+    }
+}
+
 // Position of a lane group in the CTA's item sequence (item = tt * gpt + b),
 // advanced by G items per pass without an integer division.
 struct ItemCursor {
     int tt;  // token within the CTA's range
     int b;   // item within the token, [0, gpt)
-    __device__ __forceinline__ void start(int item, int gpt)
+    __device__ __forceinline__ void start(int item, int gpt, int recip)
     {
-        tt = item / gpt;
-        b = item - tt * gpt;
+        divmod_small(item, gpt, recip, tt, b);
     }
     // dq = G / gpt, dr = G % gpt
     __device__ __forceinline__ void advance(int dq, int dr, int gpt)
@@ -296,8 +308,9 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     const int items = ntok * gpt;
 
     ItemCursor cur;
-    cur.start(grp, gpt);
-    const int dq = G / gpt, dr = G - (G / gpt) * gpt;
+    cur.start(grp, gpt, p.gpt_recip);
+    int dq, dr;
+    divmod_small(G, gpt, p.gpt_recip, dq, dr);
     for (int it0 = 0; it0 < items; it0 += G, cur.advance(dq, dr, gpt)) {  // uniform trips
         const Item m = decode_item<U>(p, tok0, cur, ntok, nbq);
 

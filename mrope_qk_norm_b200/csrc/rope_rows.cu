@@ -6,6 +6,7 @@
 // rot_dim % 16 != 0 (EXCHANGE layout) is served by a plainer kernel here that
 // passes the normalised row through shared memory to reach partners.
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <mutex>
@@ -323,6 +324,7 @@ cudaError_t launch_rope_stream(RopeParams p, int layout, int lpr, int ns, cudaSt
     p.tokens_per_cta = (int)((p.T + grid - 1) / grid);
     p.tok_base = (int)(p.T / grid);
     p.tok_rem = (int)(p.T % grid);
+    p.gpt_recip = 65536 / std::max(1, (p.Hq + u - 1) / u + (p.Hk + u - 1) / u);
     const size_t smem = ring + (size_t)p.tokens_per_cta * cs_ld * 2 * sizeof(float);
     e = launch(fn, dim3((unsigned)grid), dim3(kThreads), smem, stream, 1, p);
     if (e == cudaSuccess && rec) {
@@ -521,6 +523,10 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     p.tokens_per_cta = (int)((p.T + grid - 1) / grid);
     p.tok_base = (int)(p.T / grid);
     p.tok_rem = (int)(p.T % grid);
+    {
+        const int ug = layout == EXCHANGE ? 1 : best_u;
+        p.gpt_recip = 65536 / std::max(1, (p.Hq + ug - 1) / ug + (p.Hk + ug - 1) / ug);
+    }
 
     size_t smem = staged ? (size_t)p.tokens_per_cta * cs_ld * 2 * sizeof(float) : 0;
     if (layout == EXCHANGE)

@@ -166,9 +166,10 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     // Copy this thread's vectors of pass `pass` into ring stage `pass % S`
     // (one commit group per pass, empty past the last pass).  Passes are
     // issued in order, so the stage is a counter that wraps at S.
-    const int dq = G / gpt, dr = G - (G / gpt) * gpt;
+    int dq, dr;
+    divmod_small(G, gpt, p.gpt_recip, dq, dr);
     ItemCursor icur, ccur;  // the pass being copied in, the pass being computed
-    icur.start(grp, gpt);
+    icur.start(grp, gpt, p.gpt_recip);
     ccur = icur;
     const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(ring) + threadIdx.x * 16;
     int ist = 0, cst = 0;   // ring stage being issued into, being computed from
