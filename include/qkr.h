@@ -431,8 +431,9 @@ qkr_status qkr_launch_overlap(int32_t enable);
 /* Launch-shape override for the rope kernels, for tuning sweeps.  pipeline:
  * 0 automatic, 1 item kernel (rows straight into registers), 3 streaming
  * kernel (cp.async row ring); calls a forced kernel cannot serve fail with
- * QKR_ERR_CUDA.  heads per work item (1..4; the streaming kernel takes 1, 2 or
- * 4), tokens per CTA (1..64; kernels that stage angles cap it by their shared
+ * QKR_ERR_CUDA.  heads per work item (1..4, or 6 for GPT-J rows of 128
+ * elements with angles from a table whose rows allow 16-byte reads; the
+ * streaming kernel takes 1, 2 or 4), tokens per CTA (1..64; kernels that stage angles cap it by their shared
  * memory) and ring depth of the streaming kernel (2..4; 1 counts as 2); 0
  * keeps the automatic choice.  Process-wide; a launch racing a change on
  * another thread takes the old or the new value of each knob.  Every shape

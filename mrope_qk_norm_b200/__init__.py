@@ -168,8 +168,10 @@ def _ptr_base(t, dtype, what):
 def tune_rope(pipeline: int = 0, heads_per_item: int = 0, tokens_per_cta: int = 0,
               stages: int = 0) -> None:
     """Override the rope kernels' launch shape (0 = automatic), for tuning.
-    pipeline: 1 item kernel, 3 streaming kernel; stages: depth of the
-    streaming kernel's row ring (0 automatic, 1 and 2 both mean 2, up to 4)."""
+    pipeline: 1 item kernel, 3 streaming kernel; heads_per_item: 1 to 4, or
+    6 (GPT-J rows of 128 elements with per-item table angles only); stages:
+    depth of the streaming kernel's row ring (0 automatic, 1 and 2 both mean
+    2, up to 4)."""
     _check(_lib.qkr_tune_rope(pipeline, heads_per_item, tokens_per_cta, stages))
 
 

@@ -515,11 +515,11 @@ qkr_status qkr_tune_rope(int32_t pipeline, int32_t heads_per_item, int32_t token
                          int32_t stages)
 {
     if ((pipeline != 0 && pipeline != 1 && pipeline != 3) || heads_per_item < 0 ||
-        heads_per_item > 4 || tokens_per_cta < 0 || tokens_per_cta > 64 || stages < 0 ||
-        stages > 4)
+        (heads_per_item > 4 && heads_per_item != 6) || tokens_per_cta < 0 ||
+        tokens_per_cta > 64 || stages < 0 || stages > 4)
         return fail(QKR_ERR_INVALID_ARG,
-                    "pipeline 0, 1 or 3, heads_per_item in [0, 4], tokens_per_cta in [0, 64], "
-                    "stages in [0, 4]");
+                    "pipeline 0, 1 or 3, heads_per_item in [0, 4] or 6, tokens_per_cta in "
+                    "[0, 64], stages in [0, 4]");
     qkr::set_rope_shape_override(pipeline, heads_per_item, tokens_per_cta, stages);
     g_error.clear();
     return QKR_OK;

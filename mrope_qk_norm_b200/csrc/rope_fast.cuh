@@ -11,9 +11,10 @@
 // B200 mapping.  The op moves ~4 bytes per element and does a handful of
 // flops on it, so it is HBM-bound only if the instruction stream stays lean:
 //   * a CTA owns a balanced range of consecutive joint tokens and all of
-//     their Q and K heads; the grid is sized to the device (one wave of
-//     resident CTAs for the direct-angle kernels), so every SM gets the same
-//     share of rows and the last wave is not left half empty;
+//     their Q and K heads; the grid is sized to the device (for the
+//     direct-angle kernels, one or two waves of resident CTAs whose token
+//     count gives every lane group the same number of work items), so every
+//     SM gets the same share of rows and no pass is left part empty;
 //   * a work item is (token, Q or K, a block of U heads).  A group of LPR
 //     lanes takes an item, loads the (cos, sin) of its pairs and the gamma of
 //     its columns into registers once, and issues the 16-byte loads of all U
@@ -390,12 +391,13 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
 // the allocation decides how many CTAs share an SM and the compiler's own
 // choice moves with small code changes:
 //   * rope_fast_kernel_narrow, one 16-byte vector per lane (GPT-J rows of
-//     up to 128 elements) without the norm or with the normalised-value
-//     rounding: at least 4 CTAs per SM (64 registers; 5 for items of at
-//     most 2 heads or without the norm).  Left to itself the compiler gave
-//     these 58-77 registers.  Items of at most 2 heads with the norm stay
-//     with the compiler: bounded to 5 CTAs they ran 5% slower (GPT-J,
-//     positions, 1024 tokens);
+//     up to 128 elements) without the norm, with the normalised-value
+//     rounding, or at 6 heads per item: at least 4 CTAs per SM (64
+//     registers, no spill; 5 for items of at most 2 heads or without the
+//     norm).  Left to itself the compiler gave these 58-77 registers (76
+//     at 6 heads with the norm: 3 CTAs per SM).  Items of at most 2 heads
+//     with the norm stay with the compiler: bounded to 5 CTAs they ran 5%
+//     slower (GPT-J, positions, 1024 tokens);
 //   * rope_fast_kernel_wide, NeoX rows of three or more slots (ViT apply at
 //     D=80, 4 heads per item, ~126 registers): at least 2 CTAs per SM.  A
 //     139-register build of that shape ran at one CTA per SM, 28% slower;
@@ -428,7 +430,7 @@ constexpr KernelFn item_kernel()
     if constexpr (LAYOUT == PAIRED && NS >= 3)
         return rope_fast_kernel_wide<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>;
     else if constexpr (LAYOUT == VECTOR && NS == 1 &&
-                       (!NORM || RMODE == kRoundNormalized))
+                       (!NORM || RMODE == kRoundNormalized || U == 6))
         return rope_fast_kernel_narrow<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>;
     else
         return rope_fast_kernel<LAYOUT, LPR, NS, U, NORM, RMODE, DIRECT>;
@@ -457,6 +459,12 @@ KernelFn pick_u(int u, bool norm, int rmode)
     case 2: return pick_flags<LAYOUT, DIRECT, LPR, NS, 2>(norm, rmode);
     case 3: return pick_flags<LAYOUT, DIRECT, LPR, NS, 3>(norm, rmode);
     case 4: return pick_flags<LAYOUT, DIRECT, LPR, NS, 4>(norm, rmode);
+    case 6:
+        // one-vector GPT-J rows of 128 elements with table angles read per item
+        if constexpr (LAYOUT == VECTOR && DIRECT && LPR == 16 && NS == 1)
+            return pick_flags<LAYOUT, DIRECT, LPR, NS, 6>(norm, rmode);
+        else
+            return nullptr;
     default: return nullptr;
     }
 }

@@ -370,6 +370,57 @@ int pow2_ceil(int v)
     return p;
 }
 
+// Heads per work item (U) and tokens per CTA (tt) for one-vector GPT-J rows
+// with table angles read per item.  A CTA of tt tokens holds
+// tt * (ceil(Hq / U) + ceil(Hk / U)) work items for its lane groups, taken
+// in passes of one item per group.  The split keeps the largest share of
+// lane-group row slots that carry a row (the last pass part empty, or the
+// last item of a head set short of U heads, wastes slots), then the fewest
+// passes per CTA, then the most heads per item, over U in {4, 6} (6 only
+// for 16-lane rows; a forced U alone) and at most 3 passes.  The grid is
+// then as many such CTAs as the tokens need, usually several waves, so a
+// partly filled last wave is a small share of the launch.  Measured on B200
+// (fp32 table, head_dim 128, ~100 MB per launch; the previous rule, whole
+// passes in at most two waves, in brackets):
+//   * joint 512+4096 tokens x 24+24 heads: 6 x 2 (one pass) 19.1-19.3 us
+//     (4 x 4, three passes: 19.8); 24+24 at 4 x 1 or 4 x 2 (a quarter of the
+//     slots empty) 21.8-22.7;
+//   * 32+8 heads: 4 x 3 (30 of 32 slots) 17.9 us (22.1: 611 CTAs, one
+//     wave and 19 CTAs); 64+8: 6 x 1 18.8 (23.3: 339 CTAs); 6+6: 6 x 8
+//     18.2 (21.1); 12+12: 6 x 4 17.5 (18.2); 16+16, 28+4, 32+32, 40+8 and
+//     8+8 within 1% of the best measured shape.
+void pick_item_split(int hq, int hk, int groups, bool six, int force_u, int *u_out, int *tt_out)
+{
+    const int cand[2] = {4, 6};
+    const int ncand = force_u > 0 ? 1 : (six ? 2 : 1);
+    double best = -1.0;
+    int bu = force_u > 0 ? force_u : 4, btt = 1, bpass = 0;
+    for (int i = 0; i < ncand; ++i) {
+        const int u = force_u > 0 ? force_u : cand[i];
+        const int gpt = (hq + u - 1) / u + (hk + u - 1) / u;
+        if (gpt < 1)
+            continue;
+        const double row_share = (double)(hq + hk) / ((double)u * gpt);
+        const int ttmax = std::max(1, 3 * groups / gpt);
+        for (int tt = 1; tt <= ttmax; ++tt) {
+            const int items = tt * gpt;
+            const int passes = (items + groups - 1) / groups;
+            const double score = row_share * items / ((double)passes * groups);
+            const bool better = score > best + 1e-9 ||
+                                (score > best - 1e-9 &&
+                                 (passes < bpass || (passes == bpass && u > bu)));
+            if (better) {
+                best = score;
+                bu = u;
+                btt = tt;
+                bpass = passes;
+            }
+        }
+    }
+    *u_out = bu;
+    *tt_out = btt;
+}
+
 }  // namespace
 
 void set_rope_lanes_override(int lanes) { g_force_lpr = lanes; }
@@ -440,10 +491,12 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     // Heads per work item (U) and the token split.  Sweeps on B200 (joint
     // 512+4096 x 24 heads with both pairings, interleaved mRoPE 8192 x
     // (16+8) heads, ViT 16268 x 16 heads of D=80) gave:
-    //   * direct angles: U = 4 heads per item (U = 2 with four slots per
-    //     lane) and one wave of resident CTAs, each owning T / grid tokens.
-    //     The balanced single wave matters most: a grid that leaves a partly
-    //     filled last wave costs up to 20%;
+    //   * direct angles, one-vector GPT-J rows: U and the token split from
+    //     pick_item_split (4 or 6 heads, CTAs of one to three passes);
+    //   * direct angles, other rows: U = 4 heads per item (U = 2 with four
+    //     slots per lane) and one wave of resident CTAs, each owning T / grid
+    //     tokens.  The balanced single wave matters most there: a grid that
+    //     leaves a partly filled last wave costs up to 20%;
     //   * staged angles: U = 2 and 4 tokens per CTA (several CTAs per SM keep
     //     one CTA's staging prologue under another's row traffic).
     // Table angles are read per item by the item kernel (nothing staged) when
@@ -460,6 +513,10 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     int best_u = layout == EXCHANGE ? 1 : direct ? (ns <= 3 ? 4 : 2) : 2;
     if (g_force_u > 0 && layout != EXCHANGE)
         best_u = g_force_u;
+    // one-vector GPT-J rows with per-item table angles: U and the token split together
+    int item_tt = 0;
+    if (direct && layout == VECTOR && ns == 1 && g_force_tt <= 0)
+        pick_item_split(p.Hq, p.Hk, groups, lpr == 16, g_force_u, &best_u, &item_tt);
     const bool norm = p.norm != 0;
     const int rmode = p.round_norm;
     KernelFn fn;
@@ -480,35 +537,33 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
         const int tt = ftt < max_tt_smem ? ftt : max_tt_smem;
         grid = (p.T + tt - 1) / tt;
     } else if (direct) {
-        // Tokens per CTA: a multiple of the count that gives every lane group
-        // the same number of work items (whole passes), the smallest whose
-        // grid fits in two waves of resident CTAs for one-vector GPT-J rows
-        // and in one wave otherwise.  Joint 512+4096 tokens x 24 heads:
-        // GPT-J at 4 per CTA (1152 CTAs, 3 passes per group) 19.95 us
-        // against 20.6 us for one balanced wave of 7-8 (6 passes, the last a
-        // quarter full on the CTAs with 7) and 20.57 at 8 per CTA (one wave,
-        // whole passes); NeoX at 16 per CTA (288 CTAs, 6 passes) 21.03 us
-        // against 21.2 at 15-16 and 21.44 at 8 (two waves).  ViT apply lost
-        // 8% on two waves.
         int slots = 0;
         cudaError_t e = resident_slots(fn, 0, &slots);
         if (e != cudaSuccess)
             return e;
-        const int groups = kThreads / lpr;
-        const int items = (p.Hq + best_u - 1) / best_u + (p.Hk + best_u - 1) / best_u;
-        int a = items, b = groups;
-        while (b) {
-            const int r = a % b;
-            a = b;
-            b = r;
+        if (item_tt > 0) {
+            grid = (p.T + item_tt - 1) / item_tt;
+        } else {
+            // The other direct-angle rows (NeoX pairs, two-vector GPT-J
+            // lanes; 2 CTAs per SM): tokens per CTA a multiple of the count
+            // that gives every lane group the same number of work items
+            // (whole passes), the smallest whose grid fits in one wave of
+            // resident CTAs.  NeoX joint 512+4096 tokens x 24 heads at 16 per
+            // CTA (288 CTAs, 6 passes) 21.03 us against 21.2 at 15-16 and
+            // 21.44 at 8 (two waves); ViT apply lost 8% on two waves.
+            const int items = (p.Hq + best_u - 1) / best_u + (p.Hk + best_u - 1) / best_u;
+            int a = items, b = groups;
+            while (b) {
+                const int r = a % b;
+                a = b;
+                b = r;
+            }
+            const int64_t unit = groups / (a > 0 ? a : 1);  // tokens per CTA for whole passes
+            int64_t tt = unit;
+            if ((p.T + tt - 1) / tt > slots)
+                tt = ((p.T + slots - 1) / slots + unit - 1) / unit * unit;
+            grid = (p.T + tt - 1) / tt;
         }
-        const int64_t unit = groups / (a > 0 ? a : 1);  // tokens per CTA for whole passes
-        const int64_t waves = layout == VECTOR && ns == 1 ? 2 : 1;
-        const int64_t cap = waves * slots;
-        int64_t tt = unit;
-        if ((p.T + tt - 1) / tt > cap)
-            tt = ((p.T + cap - 1) / cap + unit - 1) / unit * unit;
-        grid = (p.T + tt - 1) / tt;
         // launches of fewer tokens than resident CTAs: one token per CTA
         // spreads them over the most SMs
         if (p.T < slots)

@@ -211,6 +211,9 @@ def test_launch_switch_refusals(qkr):
     assert L.qkr_tune_rope(3, 0, 0, 5) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(1, 0, 0, -1) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(3, 5, 0, 0) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(1, 7, 0, 0) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(1, 8, 0, 0) == qkr.QKR_ERR_INVALID_ARG
+    assert L.qkr_tune_rope(1, 6, 0, 0) == qkr.QKR_OK  # GPT-J rows of 128 with table angles
     assert L.qkr_tune_rope(3, 0, 65, 0) == qkr.QKR_ERR_INVALID_ARG
     assert L.qkr_tune_rope(0, 0, 0, 0) == qkr.QKR_OK
     assert L.qkr_launch_overlap(1) == qkr.QKR_OK

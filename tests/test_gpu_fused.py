@@ -426,13 +426,13 @@ def test_plane_sections_direct_and_staged(sections, direct):
 def test_direct_table_launch_shapes_bit_identical():
     """Every (heads per item, token split) shape of the direct-angle kernel
     computes the same bits, including ranges larger than the staged kernels
-    allow and the automatic one-wave grid."""
+    allow, 6 heads per item and the automatic split."""
     w = W.config3(seed=73, T_txt=33, img_h=6, img_w=11, H=10, D=128, pairing=W.PAIRING_GPTJ)
     cos = to_dev(torch.as_tensor(np.asarray(w.angle.cos), dtype=torch.float32))
     sin = to_dev(torch.as_tensor(np.asarray(w.angle.sin), dtype=torch.float32))
     outs = []
     try:
-        for u, tt in [(0, 0), (1, 1), (2, 3), (3, 16), (4, 64)]:
+        for u, tt in [(0, 0), (1, 1), (2, 3), (3, 16), (4, 64), (6, 5), (6, 64)]:
             qkr.tune_rope(1, u, tt)
             q, k, rec = _table_call(w, cos, sin)
             assert rec["direct_angles"] == 1
@@ -449,9 +449,9 @@ def test_direct_table_launch_shapes_bit_identical():
 
 
 def test_one_wave_grid_covers_every_token():
-    """The automatic direct-angle grid is one wave of resident CTAs with
-    balanced token ranges; token counts around multiples of the grid (and
-    fewer tokens than CTAs) still write every row exactly once."""
+    """The automatic direct-angle grid has balanced token ranges; token counts
+    around multiples of the grid (and fewer tokens than CTAs) still write
+    every row exactly once."""
     for T_txt, img_w in ((297, 1), (297, 37), (297, 45), (5, 1)):
         w = W.config3(seed=75 + img_w, T_txt=T_txt, img_h=8, img_w=img_w, H=4, D=64,
                       pairing=W.PAIRING_GPTJ)
@@ -524,12 +524,57 @@ def test_streaming_kernel_shapes_and_round_flag():
 @pytest.mark.parametrize("t_txt,img_h,img_w", [(77, 30, 21), (513, 64, 64)])
 def test_joint_ragged_token_counts(pairing, t_txt, img_h, img_w):
     """Joint launches whose token count is not a multiple of the tokens per
-    CTA the direct-angle launcher picks (whole passes per lane group: 4 for
-    GPT-J, 16 for NeoX at 24 heads), so the balanced ranges differ by one
-    token across CTAs: equal to the oracle, and every token written once."""
+    CTA the direct-angle launcher picks (2 for GPT-J at 6 heads per item, 16
+    for NeoX at 24 heads), so the balanced ranges differ by one token across
+    CTAs: equal to the oracle, and every token written once."""
     w = W.config3(seed=81, T_txt=t_txt, img_h=img_h, img_w=img_w, pairing=pairing)
     check_against_oracle(w, what="ragged joint")
     rec = qkr.last_launch()
     assert rec["direct_angles"] == 1
     assert rec["grid"] * rec["tokens_per_cta"] >= w.n_tokens
     assert (rec["grid"] - 1) * rec["tokens_per_cta"] < w.n_tokens
+
+
+def _item_split(hq, hk, groups=16):
+    """The launcher's rule for one-vector GPT-J rows with table angles, restated:
+    the largest share of lane-group row slots that carry a row, then the fewest
+    passes per CTA, then the most heads per item (4 or 6), at most 3 passes."""
+    best = None
+    for u in (4, 6):
+        gpt = -(-hq // u) + -(-hk // u)
+        share = (hq + hk) / (u * gpt)
+        for tt in range(1, max(1, 3 * groups // gpt) + 1):
+            items = tt * gpt
+            passes = -(-items // groups)
+            key = (round(share * items / (passes * groups), 9), -passes, u, -tt)
+            if best is None or key > best[0]:
+                best = (key, u, tt)
+    return best[1], best[2]
+
+
+@pytest.mark.parametrize("hq,hk", [(24, 24), (32, 8), (64, 8), (6, 6), (16, 8), (12, 12),
+                                   (40, 8), (5, 3)])
+def test_item_split_head_counts(hq, hk):
+    """One-vector GPT-J rows with table angles, over head counts for which the
+    launcher takes 4 or 6 heads per item, full or short last items and one to
+    three passes per CTA (700 joint tokens, more than one wave of resident
+    CTAs): equal to the oracle, every row written once, the documented split,
+    and bit-identical to a forced 4 heads x 4 tokens shape."""
+    cos, sin = W.joint_table(60, 20, 32, 32, 1e4)
+    A = W.AngleInputs(kind=W.ANGLE_TABLE, cos=cos.unsqueeze(0), sin=sin.unsqueeze(0))
+    w = W.random_rope_case(900 + 7 * hq + hk, [60, 640], hq, hk, 128, 128, W.PAIRING_GPTJ, A)
+    q, k, _, _ = check_against_oracle(w, what="split %d+%d" % (hq, hk))
+    rec = qkr.last_launch()
+    u, tt = _item_split(hq, hk)
+    assert rec["direct_angles"] == 1 and rec["heads_per_item"] == u, (rec, u, tt)
+    assert rec["grid"] == -(-w.n_tokens // tt), (rec, u, tt)
+    (qf, kf), rf = _with_shape(w, 1, 4, 4)
+    assert rf["heads_per_item"] == 4 and rf["tokens_per_cta"] == 4
+    assert torch.equal(q.view(torch.int16), qf.view(torch.int16))
+    assert torch.equal(k.view(torch.int16), kf.view(torch.int16))
+    for flags in (qkr.FLAG_ROUND_NORMALIZED_BF16, qkr.FLAG_EAGER_ROUNDING):
+        (qa, ka), ra = _with_shape(w, 0, flags=flags)
+        (qb, kb), rb = _with_shape(w, 1, 4, 4, flags=flags)
+        assert ra["heads_per_item"] == u and rb["heads_per_item"] == 4
+        assert torch.equal(qa.view(torch.int16), qb.view(torch.int16)), flags
+        assert torch.equal(ka.view(torch.int16), kb.view(torch.int16)), flags
