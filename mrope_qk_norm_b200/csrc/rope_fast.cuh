@@ -213,7 +213,20 @@ __device__ __forceinline__ Item decode_item(const RopeParams &p, int64_t tok0,
     return r;
 }
 
-// Joint Q/K/V: after its Q/K items a CTA copies the V rows of its tokens into
+// The 16-byte loads of an item's U rows (zero for absent heads and slots).
+template <int U, int NS>
+__device__ __forceinline__ void load_item_rows(const Item &m, const int (&vidx)[NS],
+                                               uint4 (&raw)[U][NS])
+{
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int k = 0; k < NS; ++k)
+            raw[u][k] = (u < m.nh && vidx[k] >= 0) ? ld_stream(m.src + u * m.hs + 8 * vidx[k])
+                                                   : make_uint4(0, 0, 0, 0);
+}
+
+// Joint Q/K/V: before its Q/K items a CTA copies the V rows of its tokens into
 // v_out unchanged, two rows per group at a time, with the lanes' own vector
 // slots (which cover the whole head dim in both layouts).  No math and no
 // shuffles, and a small register footprint, so the Q/K loop keeps its
@@ -271,10 +284,6 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     // Balanced ranges of at most tokens_per_cta consecutive joint tokens.
     const int64_t tok0 = cta_first_token(p);
     const int ntok = cta_tokens(p);
-    if (!DIRECT) {
-        stage_angles(p, tok0, ntok, cs_ld, cosv, sinv);
-        __syncthreads();
-    }
 
     const int lane = threadIdx.x % LPR;
     const int grp = threadIdx.x / LPR;
@@ -300,10 +309,6 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     for (int q = 0; q < NQ; ++q)
         qpair[q] = LAYOUT == PAIRED ? 8 * lane + 2 * q : 4 * (lane + LPR * (q >> 1)) + 2 * (q & 1);
 
-    // joint Q/K/V: the CTA's V rows first (plain copies), then its Q/K items
-    if (p.Hv > 0)
-        copy_v_rows<NS, LPR>(p, tok0, ntok, vidx);
-
     const int nbq = (p.Hq + U - 1) / U;
     const int gpt = nbq + (p.Hk + U - 1) / U;
     const int items = ntok * gpt;
@@ -312,17 +317,33 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     cur.start(grp, gpt, p.gpt_recip);
     int dq, dr;
     divmod_small(G, gpt, p.gpt_recip, dq, dr);
-    for (int it0 = 0; it0 < items; it0 += G, cur.advance(dq, dr, gpt)) {  // uniform trips
-        const Item m = decode_item<U>(p, tok0, cur, ntok, nbq);
+    // Staged GPT-J rows: the first item's rows are in flight while the angles
+    // are staged, so a CTA pays one memory round trip before its first
+    // rotation, not two (1024 .. 2048 tokens x 4+4 or 16+16 heads, positions:
+    // 3-19% faster).  NeoX rows keep the loads after the barrier: holding the
+    // rows across the staging took the paired kernel from 80 to 100 registers
+    // and ran 2-4% slower below 1024 tokens.
+    constexpr bool kEarlyRows = !DIRECT && LAYOUT == VECTOR;
+    Item m;
+    uint4 raw[U][NS];
+    if (kEarlyRows) {
+        m = decode_item<U>(p, tok0, cur, ntok, nbq);
+        load_item_rows<U, NS>(m, vidx, raw);
+    }
+    if (!DIRECT) {
+        stage_angles(p, tok0, ntok, cs_ld, cosv, sinv);
+        __syncthreads();
+    }
 
-        uint4 raw[U][NS];
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int k = 0; k < NS; ++k)
-                raw[u][k] = (u < m.nh && vidx[k] >= 0)
-                                ? ld_stream(m.src + u * m.hs + 8 * vidx[k])
-                                : make_uint4(0, 0, 0, 0);
+    // joint Q/K/V: the CTA's V rows first (plain copies), then its Q/K items
+    if (p.Hv > 0)
+        copy_v_rows<NS, LPR>(p, tok0, ntok, vidx);
+
+    for (int it0 = 0; it0 < items; it0 += G, cur.advance(dq, dr, gpt)) {  // uniform trips
+        if (!kEarlyRows || it0 > 0) {
+            m = decode_item<U>(p, tok0, cur, ntok, nbq);
+            load_item_rows<U, NS>(m, vidx, raw);
+        }
 
         // (cos, sin) of this lane's pairs for the item's token
         float2 C[NQ], Sn[NQ];
