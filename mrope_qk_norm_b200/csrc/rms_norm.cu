@@ -48,12 +48,22 @@ __device__ __forceinline__ float block_sum(float v, float *red)
     return t;
 }
 
+// One vector per thread (decode rows and rows up to 8192 wide): gamma is
+// loaded with x and the residual, so the row's last memory round trip is not
+// taken after the block reduction.  Wider per-thread slices load it after the
+// reduction: 4 more registers per vector would cut the large-row kernels'
+// resident CTAs.
+template <int VPT>
+constexpr bool kEarlyGamma = VPT == 1;
+
 // Loads the slice [v0, v1) of a row (vector units), forms s = bf16(x + res),
-// writes it back to residual and returns the fp32 sum of s^2 of this thread.
-// Without a residual (p.res == NULL, FP8 variant) s = x.
+// writes it back to residual and returns the fp32 sum of s^2 of this thread
+// (and, with kEarlyGamma, the slice's gamma vectors in gv).  Without a
+// residual (p.res == NULL, FP8 variant) s = x.
 template <int VPT>
 __device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v0, int v1,
-                                          float (&s)[VPT][8], bool (&live)[VPT])
+                                          float (&s)[VPT][8], bool (&live)[VPT],
+                                          uint4 (&gv)[VPT])
 {
     const __nv_bfloat16 *xr = p.x + row * p.xs;
     const bool has_res = p.res != nullptr;
@@ -65,6 +75,8 @@ __device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v
         live[k] = v < v1;
         xv[k] = live[k] ? ld_stream(xr + 8 * v) : make_uint4(0, 0, 0, 0);
         rv[k] = live[k] && has_res ? ld_stream(rr + 8 * v) : make_uint4(0, 0, 0, 0);
+        if (kEarlyGamma<VPT>)
+            gv[k] = live[k] ? ld_reuse(p.gamma + 8 * v) : make_uint4(0, 0, 0, 0);
     }
     float ss = 0.f;
 #pragma unroll
@@ -93,18 +105,19 @@ __device__ __forceinline__ float load_sum(const RmsParams &p, int64_t row, int v
 template <int VPT, bool FP8>
 __device__ __forceinline__ void scale_store(const RmsParams &p, int64_t row, int v0,
                                             float inv_rms, float (&s)[VPT][8],
-                                            const bool (&live)[VPT])
+                                            const bool (&live)[VPT], const uint4 (&gv)[VPT],
+                                            float scale)
 {
     float inv_scale = 1.f;  // y / scale is taken as y * fp32(1 / scale)
     if (FP8)
-        inv_scale = __frcp_rn(__ldg(p.scale));
+        inv_scale = __frcp_rn(kEarlyGamma<VPT> ? scale : __ldg(p.scale));
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
         if (!live[k])
             continue;
         const int v = v0 + threadIdx.x + k * blockDim.x;
         float g[8];
-        unpack8(ld_reuse(p.gamma + 8 * v), g);
+        unpack8(kEarlyGamma<VPT> ? gv[k] : ld_reuse(p.gamma + 8 * v), g);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             s[k][e] = (s[k][e] * inv_rms) * g[e];
@@ -132,12 +145,14 @@ __global__ void __launch_bounds__(kMaxThreads) rms_rows_kernel(const __grid_cons
     pdl_trigger();
     __shared__ float red[32];
     const int64_t row = blockIdx.x;
+    const float scale = FP8 && kEarlyGamma<VPT> ? __ldg(p.scale) : 1.f;
     float s[VPT][8];
     bool live[VPT];
-    const float ss = load_sum<VPT>(p, row, 0, p.hidden >> 3, s, live);
+    uint4 gv[VPT];
+    const float ss = load_sum<VPT>(p, row, 0, p.hidden >> 3, s, live, gv);
     const float total = block_sum(ss, red);
     const float inv_rms = rsqrtf(fmaf(total, p.inv_hidden, p.eps));
-    scale_store<VPT, FP8>(p, row, 0, inv_rms, s, live);
+    scale_store<VPT, FP8>(p, row, 0, inv_rms, s, live, gv, scale);
 }
 
 // One cluster per row; CTA `rank` owns vectors [rank*per, (rank+1)*per).
@@ -158,9 +173,11 @@ rms_cluster_kernel(const __grid_constant__ RmsParams p)
     const int v0 = rank * per;
     const int v1 = min(v0 + per, nvec);
 
+    const float scale = FP8 && kEarlyGamma<VPT> ? __ldg(p.scale) : 1.f;
     float s[VPT][8];
     bool live[VPT];
-    const float ss = load_sum<VPT>(p, row, v0, v1, s, live);
+    uint4 gv[VPT];
+    const float ss = load_sum<VPT>(p, row, v0, v1, s, live, gv);
     const float mine = block_sum(ss, red);
     if (threadIdx.x == 0)
         partial = mine;
@@ -170,7 +187,7 @@ rms_cluster_kernel(const __grid_constant__ RmsParams p)
         total += *cluster.map_shared_rank(&partial, r);
     cluster.barrier_arrive();  // done reading the other CTAs' shared memory
     const float inv_rms = rsqrtf(fmaf(total, p.inv_hidden, p.eps));
-    scale_store<VPT, FP8>(p, row, v0, inv_rms, s, live);
+    scale_store<VPT, FP8>(p, row, v0, inv_rms, s, live, gv, scale);
     cluster.barrier_wait();    // no CTA leaves while its partial may still be read
 }
 
