@@ -183,3 +183,32 @@ def test_rms_norm_fp8_vs_oracle(R, hidden, with_res, scale):
         assert np.array_equal(oracle.bits(res), ref_res), "residual stream not bit-exact"
     got = out8.cpu().numpy()
     assert_fp8_codes(got, ys, codes, "R=%d hidden=%d" % (R, hidden))
+
+
+@pytest.mark.parametrize("R,hidden", [(1, 5120), (7, 8192), (3, 65536)])
+def test_fp8_every_width_bit_identical(R, hidden):
+    """One vector per thread (gamma and the scale loaded with the row) and
+    several vectors per thread (loaded after the reduction), in one CTA or a
+    cluster: the same E4M3 codes and residual stream, bit for bit."""
+    w = W.config2(R=R, hidden=hidden, seed=900 + R)
+    gamma = to_dev(w.gamma)
+    sc = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    outs = []
+    try:
+        for cs, thr in [(1, 1024), (1, 256), (1, 128), (4, 512), (8, 64)]:
+            nvec = hidden // 8 // cs
+            if nvec > 8 * thr or (nvec + thr - 1) // thr > 8:
+                continue
+            qkr.tune_rms(cs, thr)
+            res = to_dev(w.residual)
+            out8 = torch.empty(R, hidden, dtype=torch.uint8, device="cuda")
+            qkr.rms_norm_fp8(to_dev(w.x), res, gamma, out8, sc, w.eps)
+            torch.cuda.synchronize()
+            info = qkr.last_launch()
+            outs.append((out8.cpu(), res.view(torch.int16).cpu(), info["slots"], info["cluster"]))
+    finally:
+        qkr.tune_rms(0, 0)
+    assert len({(o[2], o[3]) for o in outs}) >= 2, outs
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]), (o[2], o[3])
+        assert torch.equal(o[1], outs[0][1]), (o[2], o[3])
