@@ -553,7 +553,7 @@ def _item_split(hq, hk, groups=16):
 
 
 @pytest.mark.parametrize("hq,hk", [(24, 24), (32, 8), (64, 8), (6, 6), (16, 8), (12, 12),
-                                   (40, 8), (5, 3)])
+                                   (40, 8), (5, 3), (1, 1), (1, 7), (128, 8)])
 def test_item_split_head_counts(hq, hk):
     """One-vector GPT-J rows with table angles, over head counts for which the
     launcher takes 4 or 6 heads per item, full or short last items and one to
