@@ -497,8 +497,7 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     //     slots per lane) and one wave of resident CTAs, each owning T / grid
     //     tokens.  The balanced single wave matters most there: a grid that
     //     leaves a partly filled last wave costs up to 20%;
-    //   * staged angles: U = 2 and 4 tokens per CTA (several CTAs per SM keep
-    //     one CTA's staging prologue under another's row traffic).
+    //   * staged angles: U = 2 and 1-4 tokens per CTA (below).
     // Table angles are read per item by the item kernel (nothing staged) when
     // four consecutive pairs always come from one 16-byte aligned row segment
     // of one plane: aligned rows, P % 4 == 0, and no section boundary inside
@@ -568,8 +567,32 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
         // spreads them over the most SMs
         if (p.T < slots)
             grid = p.T;
-    } else {
+    } else if (layout == EXCHANGE) {
         const int tt = 4 < max_tt_smem ? 4 : max_tt_smem;
+        grid = (p.T + tt - 1) / tt;
+    } else {
+        // Staged angles: tokens per CTA that give the lane groups about one
+        // pass of work items, doubled while the grid would exceed one wave
+        // of resident CTAs, and at most 4 (several CTAs per SM keep one CTA's
+        // staging prologue under another's row traffic).  Positions launches
+        // (fp32 angles from int32 positions, B200, against 4 per CTA):
+        // GPT-J 16+16 heads x 128 at 1 per CTA, 16 / 256 tokens 2.08 / 2.75
+        // us against 3.91 / 5.46, and at 2 per CTA, 1024 tokens 5.58 against
+        // 6.86; NeoX 16+16 heads at 2 per CTA, 16 / 256 tokens 2.27 / 3.16
+        // against 3.15 / 4.22; interleaved mRoPE 16+8 heads at 2 per CTA,
+        // 64 / 512 tokens 2.04 / 2.49 against 2.55 / 2.68.  Rows of few heads
+        // (4+4 heads x 64) keep 4 per CTA.
+        int slots = 0;
+        const size_t smem4 = (size_t)4 * cs_ld * 2 * sizeof(float);
+        cudaError_t e = resident_slots(fn, smem4, &slots);
+        if (e != cudaSuccess)
+            return e;
+        const int gpt = (p.Hq + best_u - 1) / best_u + (p.Hk + best_u - 1) / best_u;
+        int tt = std::max(1, std::min(4, groups / std::max(1, gpt)));
+        while (tt < 4 && (p.T + tt - 1) / tt > slots)
+            tt = std::min(4, 2 * tt);
+        if (tt > max_tt_smem)
+            tt = max_tt_smem;
         grid = (p.T + tt - 1) / tt;
     }
     if (grid < 1)
