@@ -471,8 +471,14 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     // against 2.8.  Above it the gain is small (2457 tokens: 8.3 against
     // 8.5 us) and is lost when a streaming launch follows directly: two
     // chunks of 2457 and 5735 tokens took 24.2 us with the first on the item
-    // kernel against 23.7 us with both streaming.
-    bool stream_auto = g_force_pipe == 0 && p.angle_kind == QKR_ANGLE_POSITIONS;
+    // kernel against 23.7 us with both streaming.  With the per-head norm,
+    // launches of 8192 tokens or more take the item kernel: 8192 / 16384
+    // tokens of NeoX 16+16 heads 26.4 / 49.7 us against 30.2 / 57.7, 8+8
+    // heads 15.9 / 29.4 against 19.9 / 36.9, 32+8 heads 34.0 / 64.7 against
+    // 35.4 / 68.1, GPT-J 32+8 heads 34.8 / 65.8 against 35.8 / 70.8; 64+8
+    // heads tie.  (Below 8192 tokens the two trade places by head count.)
+    bool stream_auto = g_force_pipe == 0 && p.angle_kind == QKR_ANGLE_POSITIONS &&
+                       !(p.norm && p.T >= 8192);
     if (stream_auto && layout != EXCHANGE && g_force_tt <= 0) {
         int slots = 0;
         const cudaError_t e = stream_slots(p, layout, lpr, ns, &slots);

@@ -578,3 +578,23 @@ def test_item_split_head_counts(hq, hk):
         assert ra["heads_per_item"] == u and rb["heads_per_item"] == 4
         assert torch.equal(qa.view(torch.int16), qb.view(torch.int16)), flags
         assert torch.equal(ka.view(torch.int16), kb.view(torch.int16)), flags
+
+
+@pytest.mark.parametrize("pairing", [W.PAIRING_NEOX, W.PAIRING_GPTJ])
+def test_large_normed_positions_launch(pairing):
+    """Positions launches with the norm from 8192 tokens take the item kernel
+    (staged angles); equal to the oracle and bit-identical to the streaming
+    kernel forced on the same call."""
+    pos = np.random.default_rng(5).integers(0, 8192, (1, 8200)).astype(np.int32)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 64, 128).numpy())
+    w = W.random_rope_case(88 + pairing, [8200], 8, 8, 128, 128, pairing, A)
+    (qa, ka), ra = _with_shape(w, 0)
+    assert ra["pipelined"] == 0 and ra["direct_angles"] == 0, ra
+    (qb, kb), rb = _with_shape(w, 3)
+    assert rb["pipelined"] == 2
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(qa, rq, "large positions q")
+    assert_bf16_close(ka, rk, "large positions k")
