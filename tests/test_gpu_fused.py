@@ -598,3 +598,29 @@ def test_large_normed_positions_launch(pairing):
     rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
     assert_bf16_close(qa, rq, "large positions q")
     assert_bf16_close(ka, rk, "large positions k")
+
+
+@pytest.mark.parametrize("pairing,hq,hk,T", [(W.PAIRING_GPTJ, 16, 16, 16), (W.PAIRING_GPTJ, 16, 16, 300),
+                                             (W.PAIRING_GPTJ, 16, 16, 1024), (W.PAIRING_NEOX, 16, 16, 16),
+                                             (W.PAIRING_NEOX, 16, 8, 512), (W.PAIRING_NEOX, 4, 4, 16)])
+def test_staged_split_small_positions_launches(pairing, hq, hk, T):
+    """Positions launches below the streaming kernel's range: the staged item
+    kernel takes 1, 2 or 4 tokens per CTA (about one pass of work items, fewer
+    tokens than one wave allows); equal to the oracle and bit-identical to a
+    forced 4 tokens per CTA."""
+    pos = np.random.default_rng(T + hq).integers(0, 30000, (1, T)).astype(np.int32)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 64, 128).numpy())
+    w = W.random_rope_case(700 + T + hq, [T], hq, hk, 128, 128, pairing, A)
+    (qa, ka), ra = _with_shape(w, 0)
+    assert ra["pipelined"] == 0 and ra["direct_angles"] == 0, ra
+    assert ra["tokens_per_cta"] in (1, 2, 3, 4), ra
+    if hq + hk >= 24:
+        assert ra["tokens_per_cta"] < 4 or T > 1000, ra
+    (qb, kb), rb = _with_shape(w, 1, 2, 4)
+    assert rb["tokens_per_cta"] == 4
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(qa, rq, "staged split q")
+    assert_bf16_close(ka, rk, "staged split k")
