@@ -227,21 +227,26 @@ __device__ __forceinline__ void load_item_rows(const Item &m, const int (&vidx)[
 }
 
 // Joint Q/K/V: before its Q/K items a CTA copies the V rows of its tokens into
-// v_out unchanged, two rows per group at a time, with the lanes' own vector
+// v_out unchanged, VR rows per group at a time, with the lanes' own vector
 // slots (which cover the whole head dim in both layouts).  No math and no
-// shuffles, and a small register footprint, so the Q/K loop keeps its
-// occupancy.
-template <int NS, int LPR>
+// shuffles, and its registers are free again before the Q/K loop, so that
+// loop keeps its occupancy.  The table-path kernels keep four rows in flight:
+// joint Q/K/V 512+4096 tokens x 24 heads 29.47 -> 28.26 us (GPT-J, 3 V rows
+// per group: one round trip instead of two), 29.86 -> 29.53 us (NeoX).  The
+// kernels with staged angles keep two: there the larger copy raised the
+// register count of the small positions launches' kernel (56 -> 64) and made
+// those launches 1-3% slower.
+template <int NS, int LPR, int VR>
 __device__ __forceinline__ void copy_v_rows(const RopeParams &p, int64_t tok0, int ntok,
                                             const int (&vidx)[NS])
 {
     constexpr int G = kThreads / LPR;
     const int rows = ntok * p.Hv;
-    for (int r0 = threadIdx.x / LPR; r0 < rows; r0 += 2 * G) {
-        uint4 raw[2][NS];
-        __nv_bfloat16 *dst[2];
+    for (int r0 = threadIdx.x / LPR; r0 < rows; r0 += VR * G) {
+        uint4 raw[VR][NS];
+        __nv_bfloat16 *dst[VR];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < VR; ++j) {
             const int r = r0 + j * G;
             const bool live = r < rows;
             const int tt = live ? r / p.Hv : 0;
@@ -258,7 +263,7 @@ __device__ __forceinline__ void copy_v_rows(const RopeParams &p, int64_t tok0, i
                                                    : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int j = 0; j < VR; ++j)
 #pragma unroll
             for (int k = 0; k < NS; ++k)
                 if (dst[j] && vidx[k] >= 0)
@@ -337,7 +342,7 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
 
     // joint Q/K/V: the CTA's V rows first (plain copies), then its Q/K items
     if (p.Hv > 0)
-        copy_v_rows<NS, LPR>(p, tok0, ntok, vidx);
+        copy_v_rows<NS, LPR, DIRECT ? 4 : 2>(p, tok0, ntok, vidx);
 
     for (int it0 = 0; it0 < items; it0 += G, cur.advance(dq, dr, gpt)) {  // uniform trips
         if (!kEarlyRows || it0 > 0) {

@@ -254,7 +254,7 @@ rope_stream_kernel(const __grid_constant__ RopeParams p)
     }
     cp_async_wait(0);  // nothing is left in flight (the trailing groups are empty)
     if (p.Hv > 0)
-        copy_v_rows<NS, LPR>(p, tok0, ntok, vidx);
+        copy_v_rows<NS, LPR, 2>(p, tok0, ntok, vidx);
     pdl_exit(p.independent);
 }
 
