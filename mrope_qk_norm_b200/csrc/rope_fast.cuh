@@ -35,6 +35,10 @@
 //     GPT-J (VECTOR layout): pairs (2j, 2j+1) sit in one 32-bit word, and two
 //     words make one (A, B) float2 couple; pairs past rot_dim take (1, 0), so
 //     they pass through exactly with no branch;
+//   * NeoX rows of head_dim 64 rotated whole, with staged angles (PAIRX
+//     layout): a lane loads one vector of one rotary half and takes its
+//     partner's vector from lane l ^ rot/16 by shuffle, then runs the PAIRED
+//     arithmetic for its own half only, bit-identical to the PAIRED layout;
 //   * the fp32 sum of squares is reduced with xor shuffles inside the group;
 //     every loop trip count is uniform across a warp so the full-mask
 //     shuffles are always complete.
@@ -54,6 +58,7 @@ KernelFn pick_fast_paired_staged(int lpr, int ns, int u, bool norm, int rmode);
 KernelFn pick_fast_paired_direct(int lpr, int ns, int u, bool norm, int rmode);
 KernelFn pick_fast_vector_staged(int lpr, int ns, int u, bool norm, int rmode);
 KernelFn pick_fast_vector_direct(int lpr, int ns, int u, bool norm, int rmode);
+KernelFn pick_fast_pairx_staged(int lpr, int ns, int u, bool norm, int rmode);
 
 namespace {
 
@@ -277,8 +282,12 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     pdl_enter(p.independent);
     // Quads (couples of pairs) per lane: PAIRED lo/hi vectors hold 4, each
     // VECTOR slot holds 2.  Pass-through slots (PAIRED tail) are scaled only.
-    constexpr int NQ = RowShape<LAYOUT, NS>::NQ;
-    constexpr int NTA = RowShape<LAYOUT, NS>::NTA;
+    // A PAIRX lane rebuilds the two PAIRED slots of its pairs (its own vector
+    // and its partner's) and runs the PAIRED arithmetic on them.
+    constexpr int ML = LAYOUT == PAIRX ? PAIRED : LAYOUT;
+    constexpr int MNS = LAYOUT == PAIRX ? 2 : NS;
+    constexpr int NQ = RowShape<ML, MNS>::NQ;
+    constexpr int NTA = RowShape<ML, MNS>::NTA;
     constexpr int G = kThreads / LPR;
 
     extern __shared__ float4 smem[];
@@ -295,12 +304,18 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     const int D = p.D;
     const int nvec = D >> 3;
     const int npv = p.rot >> 4;
+    // PAIRX: the lane's pairs are those of vector hl of the first half, and
+    // its own vector is in the first half when `first`
+    const int hl = LAYOUT == PAIRX ? (lane & (npv - 1)) : lane;
+    const bool first = lane < npv;
     // vector index of each slot (-1: none)
     int vidx[NS];
 #pragma unroll
     for (int k = 0; k < NS; ++k) {
         int v;
-        if (LAYOUT == PAIRED)
+        if (LAYOUT == PAIRX)
+            v = lane;
+        else if (LAYOUT == PAIRED)
             v = k == 0 ? (lane < npv ? lane : -1)
               : k == 1 ? (lane < npv ? lane + npv : -1)
                        : 2 * npv + lane + LPR * (k - 2);
@@ -312,7 +327,8 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
     int qpair[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
-        qpair[q] = LAYOUT == PAIRED ? 8 * lane + 2 * q : 4 * (lane + LPR * (q >> 1)) + 2 * (q & 1);
+        qpair[q] = LAYOUT == PAIRED || LAYOUT == PAIRX ? 8 * hl + 2 * q
+                                                        : 4 * (lane + LPR * (q >> 1)) + 2 * (q & 1);
 
     const int nbq = (p.Hq + U - 1) / U;
     const int gpt = nbq + (p.Hk + U - 1) / U;
@@ -356,7 +372,8 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
             const bool have = LAYOUT == PAIRED ? vidx[0] >= 0 : true;
 #pragma unroll
             for (int q = 0; q < NQ; q += 2) {
-                const bool ok = m.nh > 0 && have && (LAYOUT == PAIRED || vidx[q >> 1] >= 0);
+                const bool ok = m.nh > 0 && have &&
+                                (LAYOUT == PAIRED || LAYOUT == PAIRX || vidx[q >> 1] >= 0);
                 float4 c4 = make_float4(1.f, 1.f, 1.f, 1.f);
                 float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (ok) {
@@ -378,15 +395,62 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
         if (NORM) {
             const RopeStreamDev &S = m.s1 ? p.st[1] : p.st[0];
             const __nv_bfloat16 *gam = m.isk ? S.gk : S.gq;
-            uint4 gv[NS];
+            if constexpr (LAYOUT == PAIRX) {
+                const uint4 gv[2] = {ld_reuse(gam + 8 * hl), ld_reuse(gam + 8 * (hl + npv))};
+                unpack_row<PAIRED, 2>(gv, GA, GB, GT);
+            } else {
+                uint4 gv[NS];
 #pragma unroll
-            for (int k = 0; k < NS; ++k)
-                gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
-            unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
+                for (int k = 0; k < NS; ++k)
+                    gv[k] = vidx[k] >= 0 ? ld_reuse(gam + 8 * vidx[k]) : make_uint4(0, 0, 0, 0);
+                unpack_row<LAYOUT, NS>(gv, GA, GB, GT);
+            }
         }
         RotCoef<NQ, NORM && RMODE == kRoundNone> kc;
         make_coef(kc, C, Sn, GA, GB);
 
+        if constexpr (LAYOUT == PAIRX) {
+            // this lane's half: coefficients and gammas of its own and its
+            // partner's members
+            float2 Kc[NQ], Kp[NQ], Go[NQ], Gp[NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                Kc[q] = first ? kc.K0[q] : kc.K2[q];
+                Kp[q] = first ? kc.K1[q] : kc.K3[q];
+                Go[q] = first ? GA[q] : GB[q];
+                Gp[q] = first ? GB[q] : GA[q];
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint4 own = raw[u][0];
+                uint4 par;
+                par.x = __shfl_xor_sync(0xffffffffu, own.x, npv);
+                par.y = __shfl_xor_sync(0xffffffffu, own.y, npv);
+                par.z = __shfl_xor_sync(0xffffffffu, own.z, npv);
+                par.w = __shfl_xor_sync(0xffffffffu, own.w, npv);
+                const uint4 pv[2] = {first ? own : par, first ? par : own};
+                float2 A[NQ], B[NQ], TL[NTA][4];
+                unpack_row<PAIRED, 2>(pv, A, B, TL);
+                float r = 1.f;
+                if (NORM) {
+                    // the PAIRED lane's sum over both members, reduced over
+                    // the rot/16 lanes of this half: the PAIRED order
+                    float ss = row_sumsq<PAIRED, 2>(A, B, TL);
+#pragma unroll
+                    for (int off = LPR / 4; off > 0; off >>= 1)
+                        ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    r = rsqrtf(fmaf(ss, p.inv_D, p.eps));
+                }
+                float2 O[NQ];
+                norm_rotate_half<NORM, RMODE>(A, B, r, first, Kc, Kp, Go, Gp, O);
+                uint4 outv;
+#pragma unroll
+                for (int q = 0; q < NQ; ++q)
+                    set_word(outv, q, pack2(O[q].x, O[q].y));
+                if (u < m.nh)
+                    st_stream(m.dst + (int64_t)u * D + 8 * lane, outv);
+            }
+        } else {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             float2 A[NQ], B[NQ], TL[NTA][4];
@@ -408,6 +472,7 @@ __device__ __forceinline__ void rope_fast_body(const RopeParams &p)
                     if (vidx[k] >= 0)
                         st_stream(m.dst + (int64_t)u * D + 8 * vidx[k], outv[k]);
             }
+        }
         }
     }
     pdl_exit(p.independent);
@@ -498,7 +563,13 @@ KernelFn pick_u(int u, bool norm, int rmode)
 template <int LAYOUT, bool DIRECT, int LPR>
 KernelFn pick_ns(int ns, int u, bool norm, int rmode)
 {
-    if constexpr (LAYOUT == PAIRED) {
+    if constexpr (LAYOUT == PAIRX) {
+        // head_dim 64 rotated whole: one vector per lane, 8 lanes per row
+        if constexpr (LPR == 8 && !DIRECT)
+            return ns == 1 ? pick_u<LAYOUT, DIRECT, LPR, 1>(u, norm, rmode) : nullptr;
+        else
+            return nullptr;
+    } else if constexpr (LAYOUT == PAIRED) {
         // slots 0/1: the two rotary halves of the lane's pairs; 2, 3: pass-through tail
         switch (ns) {
         case 2: return pick_u<LAYOUT, DIRECT, LPR, 2>(u, norm, rmode);

@@ -27,7 +27,7 @@
 namespace qkr {
 namespace {
 
-enum Layout { PAIRED = 0, VECTOR = 1, EXCHANGE = 2 };
+enum Layout { PAIRED = 0, VECTOR = 1, EXCHANGE = 2, PAIRX = 3 };
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -204,6 +204,44 @@ __device__ __forceinline__ void norm_rotate(
                               ? round2_bf16(__fmul2_rn(round2_bf16(__fmul2_rn(T[t][i], r2)),
                                                        GT[t][i]))
                               : __fmul2_rn(__fmul2_rn(T[t][i], r2), GT[t][i]);
+    }
+}
+
+// PAIRX layout: a lane holds one 16-byte vector of one rotary half (lane
+// l < rot/16 the first half, the others the second) and takes its partner's
+// vector from lane l ^ rot/16 by shuffle; with the two it forms the same
+// couples as a PAIRED lane and computes only its own half: a' (first half)
+// or b' (second), with the very operations norm_rotate uses for it, so the
+// results are bit-identical to the PAIRED layout's.  Kc / Kp are the lane's
+// coefficients (K0 / K1 for the first half, K2 / K3 for the second), Go / Gp
+// its own and its partner's gammas.
+template <bool NORM, int RMODE>
+__device__ __forceinline__ void norm_rotate_half(const float2 (&A)[4], const float2 (&B)[4],
+                                                 float r, bool first, const float2 (&Kc)[4],
+                                                 const float2 (&Kp)[4], const float2 (&Go)[4],
+                                                 const float2 (&Gp)[4], float2 (&O)[4])
+{
+    const float2 r2 = f2(r, r);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float2 own = first ? A[q] : B[q];
+        float2 par = first ? B[q] : A[q];
+        if (NORM && RMODE == kRoundNormalized) {
+            own = round2_bf16(__fmul2_rn(__fmul2_rn(own, r2), Go[q]));
+            par = round2_bf16(__fmul2_rn(__fmul2_rn(par, r2), Gp[q]));
+        }
+        if (NORM && RMODE == kRoundEager) {
+            own = round2_bf16(__fmul2_rn(round2_bf16(__fmul2_rn(own, r2)), Go[q]));
+            par = round2_bf16(__fmul2_rn(round2_bf16(__fmul2_rn(par, r2)), Gp[q]));
+        }
+        float2 o;
+        if (RMODE == kRoundEager)
+            o = __fadd2_rn(__fmul2_rn(own, Kc[q]), __fmul2_rn(par, Kp[q]));
+        else
+            o = __ffma2_rn(par, Kp[q], __fmul2_rn(own, Kc[q]));
+        if (NORM && RMODE == kRoundNone)
+            o = __fmul2_rn(o, r2);
+        O[q] = o;
     }
 }
 

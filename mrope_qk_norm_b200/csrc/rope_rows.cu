@@ -488,6 +488,28 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     }
     if (layout != EXCHANGE && (g_force_pipe == 3 || stream_auto))
         return launch_rope_stream(p, layout, lpr, ns, stream, rec);
+    // Table angles are read per item by the item kernel (nothing staged) when
+    // four consecutive pairs always come from one 16-byte aligned row segment
+    // of one plane: aligned rows, P % 4 == 0, and no section boundary inside
+    // a group of four pairs under a contiguous (or no) section map.
+    bool direct = layout != EXCHANGE && p.angle_kind == QKR_ANGLE_TABLE && p.tab_vec4 &&
+                  p.P % 4 == 0;
+    if (direct && p.section_mode != QKR_SECTIONS_NONE)
+        direct = p.section_mode == QKR_SECTIONS_CONTIGUOUS && p.sec[0] % 4 == 0 &&
+                 (p.sec[0] + p.sec[1]) % 4 == 0;
+    // NeoX rows of head_dim 64 rotated whole, with staged angles, take the
+    // PAIRX lane mapping: one vector per lane and the partner half by
+    // shuffle (8 lanes per row instead of 4 with two vectors each),
+    // bit-identical to the paired layout.  Positions launches of 4+4 heads:
+    // 16 / 256 / 1024 tokens 2.09 / 2.17 / 2.92 us against 2.20 / 2.27 /
+    // 3.30.  With table angles read per item it was 18-60% slower, and at
+    // head_dim 128 (16 lanes per row) slower everywhere: the per-row role
+    // selects and the partner's unpacking cost more than the occupancy gained.
+    if (layout == PAIRED && !direct && p.rot == p.D && p.rot == 64) {
+        layout = PAIRX;
+        lpr = p.rot / 8;
+        ns = 1;
+    }
     // staged (cos, sin) columns: GPT-J stages every pair of the head so pairs
     // past rot_dim rotate by the identity
     p.pw = layout == VECTOR ? p.D / 2 : p.P;
@@ -504,15 +526,6 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     //     tokens.  The balanced single wave matters most there: a grid that
     //     leaves a partly filled last wave costs up to 20%;
     //   * staged angles: U = 2 and 1-4 tokens per CTA (below).
-    // Table angles are read per item by the item kernel (nothing staged) when
-    // four consecutive pairs always come from one 16-byte aligned row segment
-    // of one plane: aligned rows, P % 4 == 0, and no section boundary inside
-    // a group of four pairs under a contiguous (or no) section map.
-    bool direct = layout != EXCHANGE && p.angle_kind == QKR_ANGLE_TABLE && p.tab_vec4 &&
-                  p.P % 4 == 0;
-    if (direct && p.section_mode != QKR_SECTIONS_NONE)
-        direct = p.section_mode == QKR_SECTIONS_CONTIGUOUS && p.sec[0] % 4 == 0 &&
-                 (p.sec[0] + p.sec[1]) % 4 == 0;
     const bool staged = !direct;
     const int max_tt_smem = staged && cs_ld > 0 ? 16384 / (8 * cs_ld) : 64;
     int best_u = layout == EXCHANGE ? 1 : direct ? (ns <= 3 ? 4 : 2) : 2;
@@ -531,6 +544,8 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     else if (layout == VECTOR)
         fn = direct ? pick_fast_vector_direct(lpr, ns, best_u, norm, rmode)
                     : pick_fast_vector_staged(lpr, ns, best_u, norm, rmode);
+    else if (layout == PAIRX)
+        fn = pick_fast_pairx_staged(lpr, ns, best_u, norm, rmode);
     else
         fn = pick_exchange(lpr, ns);
     if (!fn)
@@ -624,7 +639,7 @@ cudaError_t launch_rope_rows(const RopeParams &p_in, int pairing, cudaStream_t s
     cudaError_t err = launch(fn, dim3((unsigned)grid), dim3(kThreads), smem, stream, 1, p);
     if (err == cudaSuccess && rec) {
         *rec = LaunchRecord();
-        rec->kernel = layout == PAIRED   ? QKR_KERNEL_ROPE_PAIRED
+        rec->kernel = layout == PAIRED || layout == PAIRX ? QKR_KERNEL_ROPE_PAIRED
                     : layout == VECTOR   ? QKR_KERNEL_ROPE_VECTOR
                                          : QKR_KERNEL_ROPE_EXCHANGE;
         rec->lanes_per_row = lpr;
