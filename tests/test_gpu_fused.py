@@ -624,3 +624,28 @@ def test_staged_split_small_positions_launches(pairing, hq, hk, T):
     rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
     assert_bf16_close(qa, rq, "staged split q")
     assert_bf16_close(ka, rk, "staged split k")
+
+
+@pytest.mark.parametrize("flags", [0, qkr.FLAG_ROUND_NORMALIZED_BF16, qkr.FLAG_EAGER_ROUNDING])
+@pytest.mark.parametrize("T", [16, 300, 1024])
+def test_pairx_rows_equal_paired(flags, T):
+    """NeoX rows of head_dim 64 rotated whole with staged angles take the
+    one-vector-per-lane PAIRX mapping (8 lanes per row, the partner half by
+    shuffle): bit-identical to the streaming kernel's paired layout under
+    every rounding contract, and equal to the oracle."""
+    pos = np.random.default_rng(T).integers(0, 40000, (1, T)).astype(np.int32)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 32, 64).numpy())
+    w = W.random_rope_case(500 + T, [T], 6, 2, 64, 64, W.PAIRING_NEOX, A)
+    (qa, ka), ra = _with_shape(w, 1, flags=flags)
+    assert ra["kernel_name"] == "rope_paired" and ra["lanes_per_row"] == 8, ra
+    assert ra["slots"] == 1 and ra["pipelined"] == 0, ra
+    (qb, kb), rb = _with_shape(w, 3, flags=flags)
+    assert rb["pipelined"] == 2 and rb["lanes_per_row"] == 4, rb
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+    if flags == 0:
+        rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps,
+                                     w.angle)
+        assert_bf16_close(qa, rq, "pairx q")
+        assert_bf16_close(ka, rk, "pairx k")
