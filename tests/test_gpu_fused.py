@@ -649,3 +649,23 @@ def test_pairx_rows_equal_paired(flags, T):
                                      w.angle)
         assert_bf16_close(qa, rq, "pairx q")
         assert_bf16_close(ka, rk, "pairx k")
+
+
+@pytest.mark.parametrize("streams_T", [[1], [5, 37], [64, 700]])
+def test_pairx_joint_streams_and_edges(streams_T):
+    """The one-vector-per-lane NeoX mapping on joint launches (text then
+    image stream, positions over the joint tokens) and a single token: equal
+    to the oracle and bit-identical to the paired streaming kernel."""
+    T = sum(streams_T)
+    pos = np.random.default_rng(T + 3).integers(0, 9000, (1, T)).astype(np.int32)
+    A = W.AngleInputs(kind=W.ANGLE_POSITIONS, positions=pos,
+                      inv_freq=W.inv_freq(1e4, 32, 64).numpy())
+    w = W.random_rope_case(600 + T, streams_T, 5, 3, 64, 64, W.PAIRING_NEOX, A)
+    (qa, ka), ra = _with_shape(w, 1)
+    assert ra["lanes_per_row"] == 8 and ra["slots"] == 1, ra
+    (qb, kb), _ = _with_shape(w, 3)
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+    rq, rk = oracle.qk_norm_rope(w.streams, w.Hq, w.Hk, w.D, w.rot, w.pairing, w.eps, w.angle)
+    assert_bf16_close(qa, rq, "pairx joint q")
+    assert_bf16_close(ka, rk, "pairx joint k")
