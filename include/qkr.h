@@ -397,7 +397,9 @@ enum {
 typedef struct qkr_launch_info {
     int32_t kernel;          /* QKR_KERNEL_* */
     int32_t lanes_per_row;   /* rope kernels: lanes that share one head row */
-    int32_t slots;           /* rope: 16-byte vectors per lane per row; rms: per thread */
+    int32_t slots;           /* rope: 16-byte vectors per lane per row (NeoX rows of
+                                head_dim 64 with staged angles: 1, the lane taking its
+                                partner half from another lane); rms: per thread */
     int32_t tokens_per_cta;  /* rope / vit: tokens one CTA covers */
     int32_t heads_per_item;  /* rope: head rows of one token a lane group loads
                                 together */
